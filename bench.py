@@ -1,0 +1,410 @@
+#!/usr/bin/env python
+"""Benchmark of the Spense hybrid 2:4-sparse + dense FP8 GEMM on B200.
+
+Workload (default): the attention projections of a 32B-class decoder (hidden
+5120): q_proj 8192x5120, k_proj and v_proj 1024x5120, o_proj 5120x8192, FP8
+e4m3 weights with the last 25% of the input columns dense, M = 16 decode
+tokens. One step = the four GEMMs of one layer. Eight layers' packed weights
+(542 MB, more than the 126 MB L2) are rotated so every step streams its
+weights from HBM. Inputs are seeded synthetic tensors (no model weights).
+
+Metric: weight-stream GB/s = algorithmic bytes (packed values + 2-bit
+metadata + dense columns + scales + activations + bf16 output) / time; also
+the speedup over the same kernel on the dense FP8 matrix (dense_frac = 1).
+
+Prints one JSON line (rank 0). Multi-GPU runs are independent replicas (the
+GEMM has no exchange step), launched one process per GPU.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["spense", "reference"], default="spense")
+    ap.add_argument("--tokens", type=int, default=16, help="decode tokens M")
+    ap.add_argument("--layers", type=int, default=8, help="weight sets rotated between steps")
+    ap.add_argument("--dense-frac", type=float, default=0.25)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+SHAPES = (("q_proj", 8192, 5120), ("k_proj", 1024, 5120), ("v_proj", 1024, 5120), ("o_proj", 5120, 8192))
+
+
+def workload_config(args):
+    return {
+        "workload": f"attn32b q/k/v/o projections, decode M={args.tokens}",
+        "shapes": [f"{n}x{k}" for _, n, k in SHAPES],
+        "tokens": args.tokens,
+        "dense_frac": args.dense_frac,
+        "dense_columns": "tail (SpenseGPT)",
+        "weights": "FP8 e4m3 N(0,0.02) per-channel absmax scales; X N(0,1) per-token scales; seed 1",
+        "l2": f"{args.layers} weight sets rotated per step (inputs larger than L2)",
+    }
+
+
+def step_bytes(args, Kd_of):
+    from dense_fp8_gemm_b200 import workloads
+    return sum(workloads.algorithmic_bytes(n, k, Kd_of(k), args.tokens) for _, n, k in SHAPES)
+
+
+def kd_of(args):
+    from dense_fp8_gemm_b200 import workloads
+    return lambda k: workloads.dense_count(k, args.dense_frac)
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+
+
+def oracle_sample_rate(args, rows_per_shape: int, budget_s: float, nthreads: int):
+    """Times the CPU oracle (as it stands) on `rows_per_shape` rows of each
+    projection, repeating until `budget_s` elapses. Returns (GB/s, seconds, reps)."""
+    import oracle
+    from dense_fp8_gemm_b200 import workloads
+    wl = workloads.ATTN32B
+    items = []
+    for i, (_, n, k) in enumerate(SHAPES):
+        w = workloads.make_weight(wl, i, args.dense_frac)
+        rows = np.linspace(0, n - 1, rows_per_shape).astype(np.int64)
+        keep = oracle.pack(w.W[rows], Kd=w.Kd)["keep"]
+        X, s_x = workloads.make_activations(wl, i, args.tokens)
+        items.append((X, s_x, w.W[rows].copy(), w.s_w[rows].copy(), keep, k, w.Kd))
+    byts = sum(workloads.algorithmic_bytes(rows_per_shape, k, kd, args.tokens) for *_, k, kd in items)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        for X, s_x, W, s_w, keep, _, _ in items:
+            oracle.gemm(X, s_x, W, s_w, keep=keep, nthreads=nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return byts * reps / el / 1e9, el, reps, byts
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cores = os.cpu_count() or 1
+    rows = 32  # bounded sample per step: 32 output rows of each projection
+    done_bytes = 0
+    import oracle as _o
+    from dense_fp8_gemm_b200 import workloads as _w
+    wl = _w.ATTN32B
+    items = []
+    for i, (_, n, k) in enumerate(SHAPES):
+        w = _w.make_weight(wl, i, args.dense_frac)
+        r = np.linspace(0, n - 1, rows).astype(np.int64)
+        keep = _o.pack(w.W[r], Kd=w.Kd)["keep"]
+        X, s_x = _w.make_activations(wl, i, args.tokens)
+        items.append((X, s_x, w.W[r].copy(), w.s_w[r].copy(), keep, k, w.Kd))
+    per_step = sum(_w.algorithmic_bytes(rows, k, kd, args.tokens) for *_, k, kd in items)
+    for _ in range(args.warmup):
+        for X, s_x, W, s_w, keep, _, _ in items:
+            _o.gemm(X, s_x, W, s_w, keep=keep, nthreads=cores)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        for X, s_x, W, s_w, keep, _, _ in items:
+            _o.gemm(X, s_x, W, s_w, keep=keep, nthreads=cores)
+        done_bytes += per_step
+    el = time.perf_counter() - t0
+    value = done_bytes / el / 1e9
+    sample = f"{rows} rows of each of q/k/v/o per step (M={args.tokens}); full rows scale linearly"
+    line = {
+        "impl": "reference", "metric": "spense_fp8_weight_stream_GBps", "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el / max(1, args.steps) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(args),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- Spense arm
+
+
+def run_spense(args):
+    import torch
+    import torch.distributed as dist
+
+    from dense_fp8_gemm_b200 import spense, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    M = args.tokens
+    Kd_of = kd_of(args)
+    wl = workloads.ATTN32B
+    # ---- weights: one synthetic layer, packed into `layers` distinct buffer sets
+    layers_sp, layers_dn, dims = [], [], []
+    host_w = []
+    for i, (_, n, k) in enumerate(SHAPES):
+        w = workloads.make_weight(wl, i, args.dense_frac)
+        host_w.append(w)
+        dims.append((n, k, w.Kd))
+    for _ in range(args.layers):
+        sp, dn = [], []
+        for w in host_w:
+            Wd = torch.from_numpy(w.W).to(dev)
+            sd = torch.from_numpy(w.s_w).to(dev)
+            sp.append(spense.pack(Wd, sd, Kd=w.Kd))
+            dn.append(spense.pack(Wd, sd, Kd=w.K))
+            del Wd
+        layers_sp.append(sp)
+        layers_dn.append(dn)
+    acts = []
+    for i in range(len(SHAPES)):
+        X, s_x = workloads.make_activations(wl, i, M)
+        acts.append((torch.from_numpy(X).to(dev), torch.from_numpy(s_x).to(dev), X, s_x))
+    Ys = [torch.empty((M, n), dtype=torch.bfloat16, device=dev) for n, _, _ in dims]
+    ws_bytes = max(spense.workspace_size(p, M) for L in (layers_sp, layers_dn) for p in L[0])
+    ws = spense.new_workspace(ws_bytes, dev)
+    torch.cuda.synchronize()
+
+    def launch_layer(layer_packs):
+        for s, pw in enumerate(layer_packs):
+            spense.gemm(pw, acts[s][0], acts[s][1], Ys[s], ws, stream)
+
+    def capture(layer_list, with_events=False):
+        graphs, evs = [], []
+        for L in layer_list:
+            launch_layer(L)  # warm (attribute setup outside capture)
+        torch.cuda.synchronize()
+        for L in layer_list:
+            g = torch.cuda.CUDAGraph()
+            e = [(torch.cuda.Event(enable_timing=True, external=True),
+                  torch.cuda.Event(enable_timing=True, external=True)) for _ in L] if with_events else None
+            with torch.cuda.graph(g):
+                for s, pw in enumerate(L):
+                    if with_events:
+                        e[s][0].record()
+                    spense.gemm(pw, acts[s][0], acts[s][1], Ys[s], ws, torch.cuda.current_stream())
+                    if with_events:
+                        e[s][1].record()
+            graphs.append(g)
+            evs.append(e)
+        torch.cuda.synchronize()
+        return graphs, evs
+
+    def timed(graphs, steps, warmup):
+        for i in range(warmup):
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(steps):
+            graphs[i % len(graphs)].replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1) / 1e3  # seconds
+
+    g_sp, _ = capture(layers_sp)
+    g_dn, _ = capture(layers_dn)
+
+    with ClockSampler(local) as clocks:
+        t_sp = timed(g_sp, args.steps, args.warmup)
+    t_dn = timed(g_dn, args.steps, args.warmup)
+
+    if world > 1:
+        t = torch.tensor([t_sp, t_dn], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_sp, t_dn = t.tolist()
+
+    per_step = step_bytes(args, Kd_of)
+    value = per_step * args.steps * world / t_sp / 1e9
+    launches = args.steps * len(SHAPES)
+
+    # ---- dominant kernel: per-launch device time from events captured around each GEMM
+    g_ev, evs = capture(layers_sp, with_events=True)
+    dur = [[] for _ in SHAPES]
+    reps = max(8, min(args.steps, 64))
+    for i in range(reps):
+        g_ev[i % len(g_ev)].replay()
+        torch.cuda.synchronize()
+        for s, (a, b) in enumerate(evs[i % len(g_ev)]):
+            dur[s].append(a.elapsed_time(b) / 1e3)
+    per_launch = [statistics.median(d) for d in dur]
+    bytes_per_launch = [workloads.algorithmic_bytes(n, k, kd, M) for n, k, kd in dims]
+    achieved = sum(bytes_per_launch) / sum(per_launch) / 1e9
+    peak, peak_kind = read_peaks()
+    del g_ev, evs
+
+    # ---- e2e through the host-buffer entry point (copies inside the timed region)
+    hws = spense.new_workspace(max(spense.host_workspace_size(p, M) for p in layers_sp[0]), dev)
+    hx = [torch.from_numpy(a[2]).pin_memory() for a in acts]
+    hs = [torch.from_numpy(a[3]).pin_memory() for a in acts]
+    hy = [torch.empty((M, n), dtype=torch.bfloat16).pin_memory() for n, _, _ in dims]
+    e2e_steps = max(4, min(args.steps, 100))
+    for i in range(min(args.warmup, 4)):
+        for s, pw in enumerate(layers_sp[i % args.layers]):
+            spense.gemm_host(pw, hx[s], hs[s], hy[s], hws, stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        for s, pw in enumerate(layers_sp[i % args.layers]):
+            spense.gemm_host(pw, hx[s], hs[s], hy[s], hws, stream)
+    e1.record()
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_e2e = t.item()
+    h2d = sum(M * k + 4 * M for _, k, _ in dims)
+    d2h = sum(2 * M * n for n, _, _ in dims)
+    e2e_value = per_step * e2e_steps * world / t_e2e / 1e9
+
+    status = spense.workspace_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status word {status:#x}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        gbs, el, reps_c, byts = oracle_sample_rate(args, 256, args.cpu_seconds, cores)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"256 rows of each of q/k/v/o, M={args.tokens}, {reps_c} passes in {el:.1f} s"}
+
+    if rank == 0:
+        tflops = sum(workloads.useful_flops(n, k, kd, M) for n, k, kd in dims) * args.steps * world / t_sp / 1e12
+        line = {
+            "metric": "spense_fp8_weight_stream_GBps", "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_sp / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe4m3->f32",
+            "data": "synthetic", "config": workload_config(args),
+            "speedup_vs_dense_fp8": t_dn / t_sp,
+            "dense_fp8_GBps": (sum(workloads.algorithmic_bytes(n, k, k, M) for n, k, _ in dims)
+                               * args.steps * world / t_dn / 1e9),
+            "tflops": tflops,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
+                         "kernel": "spense_gemm_kernel",
+                         "per_launch_us": {SHAPES[s][0]: per_launch[s] * 1e6 for s in range(len(SHAPES))}},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+
+    for L in layers_sp + layers_dn:
+        for p in L:
+            p.free()
+    if world > 1:
+        dist.barrier()
+        del g_sp, g_dn
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_spense(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

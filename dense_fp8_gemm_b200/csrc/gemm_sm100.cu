@@ -1,0 +1,382 @@
+// Hybrid 2:4-sparse + dense FP8 weight GEMM for sm_100a:
+//   Y[m][n] = bf16(s_x[m] * s_w[n] * (sum over the 2:4 region + sum over the dense region))
+//
+// Page: "SpenseGPT: Practical One-shot Pruning Enabling Sparse and Dense GEMMs
+// for LLM Inference" (gist.science technical summary), Technical Summary §2.A:
+// the input-split execution runs the sparse GEMM over the first part of the
+// input dimension and the dense GEMM over the second, with accumulation. Here
+// both phases feed ONE fp32 accumulator in tensor memory inside one kernel:
+// tcgen05.mma.sp over the 2:4 blocks, then tcgen05.mma over the dense blocks.
+//
+// Layout of the work (swap-AB): weight rows are the MMA M dimension (128 per
+// tile), tokens are the MMA N dimension (padded to a multiple of 16), K is the
+// packed column order (2:4 region first, then the dense region).
+//
+// Roles (one CTA per SM, 192 threads):
+//   warp 0   producer: bulk copies of the packed weight blocks (values,
+//            metadata, dense columns) and 2-D TMA loads of the activation tile
+//            into a ring of shared-memory stages;
+//   warp 1   allocates tensor memory; one lane copies the metadata into tensor
+//            memory (tcgen05.cp) and issues the MMAs;
+//   warps 2-5 epilogue: tensor memory -> registers, scales, bf16 stores, or
+//            fp32 partials plus a deterministic fix-up when a tile is shared.
+//
+// Work split ("stream-K by bytes"): the blocks of all tiles form one sequence,
+// each block weighted by the HBM bytes it streams (a 2:4 block 20 KiB, a dense
+// block 16 KiB). CTA g takes the blocks whose start falls in
+// [g T / G, (g+1) T / G) of the total weight T. A tile split across CTAs is
+// finished by the last CTA to arrive, which sums every contributor's partial in
+// CTA order, so the result does not depend on arrival order.
+//
+// Every wait is bounded (1.5 s by %globaltimer); on expiry the kernel records a
+// code in the workspace status word and all roles leave their loops.
+#include <algorithm>
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "sm100_ptx.cuh"
+#include "spense_internal.h"
+
+namespace spense {
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 1500000000ull;
+
+struct alignas(8) Barriers {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  int abort_flag;
+  int fix_flag;
+};
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, unsigned int* status,
+                                         unsigned int code, volatile int* abort_flag) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  uint32_t it = 0;
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((++it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        atomicOr(status, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- work split
+struct Split {
+  const GemmParams& p;
+  int nblk;
+  __device__ explicit Split(const GemmParams& pp) : p(pp), nblk(pp.nsb + pp.ndb) {}
+
+  // Start weight of block j inside a tile.
+  __device__ long long block_start(int j) const {
+    return j <= p.nsb ? static_cast<long long>(kCostSparse) * j
+                      : static_cast<long long>(kCostSparse) * p.nsb +
+                            static_cast<long long>(kCostDense) * (j - p.nsb);
+  }
+  // First linear block (tile * nblk + j) whose start weight is >= c.
+  __device__ long long first_block_at(long long c) const {
+    const long long t = c / p.tile_cost;
+    const long long r = c - t * p.tile_cost;
+    const long long sp = static_cast<long long>(kCostSparse) * p.nsb;
+    long long j;
+    if (r <= sp)
+      j = (r + kCostSparse - 1) / kCostSparse;
+    else
+      j = p.nsb + (r - sp + kCostDense - 1) / kCostDense;
+    return t * nblk + j;
+  }
+  __device__ long long cta_start_weight(int g) const {
+    return (static_cast<long long>(g) * p.total_cost + p.grid - 1) / p.grid;
+  }
+  __device__ long long cta_first_block(int g) const { return first_block_at(cta_start_weight(g)); }
+  // CTA owning block j of tile t.
+  __device__ int owner(long long t, int j) const {
+    const long long s = t * p.tile_cost + block_start(j);
+    return static_cast<int>((s * p.grid) / p.total_cost);
+  }
+  // Partial slot CTA g uses for tile t: 0 for its first tile, 1 for its last.
+  __device__ int slot(int g, long long t) const { return (cta_first_block(g) / nblk == t) ? 0 : 1; }
+};
+
+// Iterates the units (t, j0, j1) of a block range.
+struct UnitIter {
+  long long b, b1;
+  int nblk;
+  __device__ UnitIter(long long b0_, long long b1_, int nblk_) : b(b0_), b1(b1_), nblk(nblk_) {}
+  __device__ bool next(long long& t, int& j0, int& j1) {
+    if (b >= b1) return false;
+    t = b / nblk;
+    j0 = static_cast<int>(b - t * nblk);
+    const long long left = b1 - b;
+    j1 = static_cast<int>(left < nblk - j0 ? j0 + left : nblk);
+    b += j1 - j0;
+    return true;
+  }
+};
+
+__device__ __forceinline__ uint16_t to_bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    spense_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < p.stages; ++s) {
+      ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), 128);
+    }
+    bars->abort_flag = 0;
+    bars->fix_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) ptx::prefetch_tensormap(&tmap_x);
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), p.tmem_cols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const Split split(p);
+  const long long b0 = split.cta_first_block(g);
+  const long long b1 = split.cta_first_block(g + 1);
+  const uint32_t smem_base = ptx::smem_addr(smem);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = ptx::policy_evict_first();
+      const uint64_t pol_x = ptx::policy_evict_last();
+      UnitIter units(b0, b1, split.nblk);
+      long long t;
+      int j0, j1;
+      uint32_t it = 0;
+      bool ok = true;
+      while (ok && units.next(t, j0, j1)) {
+        const long long n_tile = t / p.m_tiles;
+        const int y0 = static_cast<int>(t % p.m_tiles) * kMaxTokenTile;
+        for (int j = j0; j < j1; ++j, ++it) {
+          const uint32_t s = it % p.stages;
+          const uint32_t ph = (it / p.stages) & 1u;
+          if (!wait_bar(ptx::smem_addr(&bars->empty[s]), ph ^ 1u, p.status,
+                        SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_s = smem_base + s * p.stage_bytes;
+          const uint32_t b_s = a_s + kBlockBytes;
+          const uint32_t e_s = b_s + p.b_bytes;
+          const uint32_t full = ptx::smem_addr(&bars->full[s]);
+          const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
+          if (j < p.nsb) {
+            const size_t blk = static_cast<size_t>(n_tile) * p.nsb + j;
+            ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * box);
+            ptx::bulk_g2s(a_s, p.vs_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
+            ptx::bulk_g2s(e_s, p.e_t + blk * kMetaBlockBytes, kMetaBlockBytes, full, pol_w);
+            ptx::tma_load_2d(b_s, &tmap_x, j * kSparseBlockCols, y0, full, pol_x);
+            ptx::tma_load_2d(b_s + box, &tmap_x, j * kSparseBlockCols + 128, y0, full, pol_x);
+          } else {
+            const int jd = j - p.nsb;
+            const size_t blk = static_cast<size_t>(n_tile) * p.ndb + jd;
+            ptx::mbar_arrive_expect_tx(full, kBlockBytes + box);
+            ptx::bulk_g2s(a_s, p.wd_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
+            ptx::tma_load_2d(b_s, &tmap_x, p.Ks + jd * kDenseBlockCols, y0, full, pol_x);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc_sp = ptx::idesc_f8(static_cast<uint32_t>(p.npad), true);
+      const uint32_t idesc_d = ptx::idesc_f8(static_cast<uint32_t>(p.npad), false);
+      const uint32_t e_col0 = static_cast<uint32_t>(p.nacc * p.npad);
+      UnitIter units(b0, b1, split.nblk);
+      long long t;
+      int j0, j1;
+      uint32_t it = 0, u = 0, ebuf = 0;
+      bool ok = true;
+      while (ok && units.next(t, j0, j1)) {
+        const uint32_t acc = u % p.nacc;
+        const uint32_t aph = (u / p.nacc) & 1u;
+        if (!wait_bar(ptx::smem_addr(&bars->acc_empty[acc]), aph ^ 1u, p.status,
+                      SPENSE_DEVICE_TIMEOUT_MMA, abort_flag)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.npad);
+        for (int j = j0; j < j1; ++j, ++it) {
+          const uint32_t s = it % p.stages;
+          const uint32_t ph = (it / p.stages) & 1u;
+          if (!wait_bar(ptx::smem_addr(&bars->full[s]), ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
+                        abort_flag)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t a_s = smem_base + s * p.stage_bytes;
+          const uint32_t b_s = a_s + kBlockBytes;
+          const uint32_t e_s = b_s + p.b_bytes;
+          const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
+          if (j < p.nsb) {
+            const uint32_t e_tmem = tmem_base + e_col0 + ebuf * 8u;
+            ptx::tmem_cp_128x128b(e_tmem, ptx::desc_rows16(e_s));
+            ptx::tmem_cp_128x128b(e_tmem + 4u, ptx::desc_rows16(e_s + 2048u));
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+              const uint64_t ad = ptx::desc_sw128(a_s + 32u * k);
+              const uint64_t bd = ptx::desc_sw128(b_s + (k >> 1) * box + (k & 1u) * 64u);
+              ptx::mma_sp_f8(d_tmem, ad, bd, e_tmem + 2u * k, idesc_sp,
+                             (j > j0 || k > 0) ? 1u : 0u);
+            }
+            ebuf ^= 1u;
+          } else {
+#pragma unroll
+            for (uint32_t k = 0; k < 4; ++k) {
+              const uint64_t ad = ptx::desc_sw128(a_s + 32u * k);
+              const uint64_t bd = ptx::desc_sw128(b_s + 32u * k);
+              ptx::mma_f8(d_tmem, ad, bd, idesc_d, (j > j0 || k > 0) ? 1u : 0u);
+            }
+          }
+          ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
+        }
+        if (!ok) break;
+        ptx::mma_commit(ptx::smem_addr(&bars->acc_full[acc]));
+        ++u;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int et = threadIdx.x - 64;           // 0..127
+    const int quarter = warp & 3;              // tensor-memory lane quarter this warp may read
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    UnitIter units(b0, b1, split.nblk);
+    long long t;
+    int j0, j1;
+    uint32_t u = 0;
+    while (units.next(t, j0, j1)) {
+      const uint32_t acc = u % p.nacc;
+      const uint32_t aph = (u / p.nacc) & 1u;
+      const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
+                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
+      ptx::tc_fence_after();
+      const long long n_tile = t / p.m_tiles;
+      const int m0 = static_cast<int>(t % p.m_tiles) * kMaxTokenTile;
+      const int m_valid = min(p.npad, p.M - m0);
+      const int n = static_cast<int>(n_tile) * kTileRows + row;
+      const bool row_ok = n < p.N;
+      const float sw = row_ok ? __ldg(p.s_w + n) : 0.0f;
+      const bool whole = (j0 == 0 && j1 == split.nblk);
+      const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
+      float* part = nullptr;
+      if (!whole)
+        part = p.partials + (static_cast<size_t>(g) * 2 + split.slot(g, t)) * p.npad * kTileRows;
+      for (int c0 = 0; c0 < m_valid; c0 += 16) {
+        uint32_t v[16];
+        ptx::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), v);
+        ptx::tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int m = c0 + i;
+          if (m < m_valid) {
+            const float a = __uint_as_float(v[i]);
+            if (whole) {
+              if (row_ok)
+                p.y[static_cast<size_t>(m0 + m) * p.N + n] =
+                    to_bf16_bits(a * sw * __ldg(p.s_x + m0 + m));
+            } else {
+              part[static_cast<size_t>(m) * kTileRows + row] = a;
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
+      ++u;
+      if (!whole) {
+        __threadfence();
+        ptx::named_bar_sync(1, 128);
+        const int g_lo = split.owner(t, 0);
+        const int g_hi = split.owner(t, split.nblk - 1);
+        if (et == 0) {
+          const unsigned int old = atomicAdd(p.counters + t, 1u);
+          bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
+        }
+        ptx::named_bar_sync(1, 128);
+        const int finisher = *reinterpret_cast<volatile int*>(&bars->fix_flag);
+        if (finisher) {
+          __threadfence();
+          for (int m = 0; m < m_valid; ++m) {
+            float sum = 0.0f;
+            for (int gg = g_lo; gg <= g_hi; ++gg) {
+              const float* pp =
+                  p.partials + (static_cast<size_t>(gg) * 2 + split.slot(gg, t)) * p.npad * kTileRows;
+              sum += __ldcg(pp + static_cast<size_t>(m) * kTileRows + row);
+            }
+            if (row_ok)
+              p.y[static_cast<size_t>(m0 + m) * p.N + n] = to_bf16_bits(sum * sw * __ldg(p.s_x + m0 + m));
+          }
+          if (et == 0) atomicExch(p.counters + t, 0u);
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace
+
+uint32_t gemm_max_smem() { return 232448u; }
+
+cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t smem_bytes,
+                        cudaStream_t stream) {
+  static thread_local int configured_for = -1;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  if (configured_for != dev) {
+    st = cudaFuncSetAttribute(spense_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(gemm_max_smem()));
+    if (st != cudaSuccess) return st;
+    configured_for = dev;
+  }
+  spense_gemm_kernel<<<p.grid, kGemmThreads, smem_bytes, stream>>>(tmap_x, p);
+  return cudaGetLastError();
+}
+
+}  // namespace spense

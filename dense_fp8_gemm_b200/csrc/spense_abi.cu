@@ -1,0 +1,442 @@
+// Host side of the Spense C ABI: argument validation, the packed handle,
+// launch planning (tile, token padding, stream-K grid, pipeline depth), the
+// activation tensor map, and the workspace layout.
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include <cudaTypedefs.h>
+
+#include "spense_internal.h"
+
+using namespace spense;
+
+struct spense_packed {
+  int device = -1;
+  int64_t N = 0, K = 0, Ks = 0, Kd = 0;
+  int n_tiles = 0, nsb = 0, ndb = 0;
+  uint8_t* vs_t = nullptr;
+  uint8_t* e_t = nullptr;
+  uint8_t* wd_t = nullptr;
+  float* s_w = nullptr;
+  int32_t* perm = nullptr;
+  uint8_t* vs_c = nullptr;
+  uint8_t* e_c = nullptr;
+  uint8_t* wd_c = nullptr;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+spense_status fail(spense_status code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+spense_status ok() {
+  g_last_error.clear();
+  return SPENSE_OK;
+}
+
+spense_status cuda_fail(cudaError_t e, const char* what) {
+  if (e == cudaErrorMemoryAllocation)
+    return fail(SPENSE_ERR_OOM, "%s: %s", what, cudaGetErrorString(e));
+  return fail(SPENSE_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct DeviceInfo {
+  int major = 0;
+  int sms = 0;
+};
+
+// Current device's capability and SM count (cached per device).
+spense_status current_device(int* dev, DeviceInfo* info) {
+  static std::mutex mu;
+  static std::vector<DeviceInfo> cache;
+  cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess) return fail(SPENSE_ERR_UNSUPPORTED, "no CUDA device: %s", cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<int>(cache.size()) <= *dev) cache.resize(*dev + 1);
+  DeviceInfo& d = cache[*dev];
+  if (d.sms == 0) {
+    if (cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess) {
+      d.sms = 0;
+      return fail(SPENSE_ERR_UNSUPPORTED, "cannot query device %d", *dev);
+    }
+  }
+  *info = d;
+  if (d.major != 10)
+    return fail(SPENSE_ERR_UNSUPPORTED, "device %d has compute capability %d.x; sm_100 is required",
+                *dev, d.major);
+  return SPENSE_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+void free_handle(spense_packed* h) {
+  if (h == nullptr) return;
+  for (void* p : {static_cast<void*>(h->vs_t), static_cast<void*>(h->e_t), static_cast<void*>(h->wd_t),
+                  static_cast<void*>(h->s_w), static_cast<void*>(h->perm), static_cast<void*>(h->vs_c),
+                  static_cast<void*>(h->e_c), static_cast<void*>(h->wd_c)})
+    if (p != nullptr) cudaFree(p);
+  delete h;
+}
+
+// Launch plan for (handle, M) on a device with `sms` SMs.
+GemmPlan make_plan(const spense_packed* h, int64_t M, int sms) {
+  GemmPlan pl{};
+  pl.npad = M > kMaxTokenTile ? kMaxTokenTile : static_cast<int>(round_up(static_cast<size_t>(M), 16));
+  pl.m_tiles = static_cast<int>((M + kMaxTokenTile - 1) / kMaxTokenTile);
+  pl.n_tiles = h->n_tiles;
+  pl.tiles = pl.n_tiles * pl.m_tiles;
+  pl.nsb = h->nsb;
+  pl.ndb = h->ndb;
+  pl.tile_cost = kCostSparse * pl.nsb + kCostDense * pl.ndb;
+  pl.total_cost = static_cast<long long>(pl.tiles) * pl.tile_cost;
+  // At least one maximal block of weight per CTA, so no CTA owns an empty range.
+  long long grid = pl.total_cost / kCostSparse;
+  grid = std::max<long long>(1, std::min<long long>(grid, sms));
+  pl.grid = static_cast<int>(grid);
+  pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.nsb > 0 ? 256u : 128u);
+  pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.nsb > 0 ? kMetaBlockBytes : 0);
+  const uint32_t reserve = 1024 + 512;  // alignment slack + barriers
+  pl.stages = static_cast<int>(std::min<uint32_t>(kMaxStages, (gemm_max_smem() - reserve) / pl.stage_bytes));
+  pl.nacc = (2 * pl.npad + 16 <= 512) ? 2 : 1;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(pl.nacc * pl.npad + 16)) cols <<= 1;
+  pl.tmem_cols = cols;
+  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
+
+  WorkspaceLayout& w = pl.ws;
+  size_t off = 256;  // header: status word
+  w.counters_off = off;
+  w.counters_bytes = round_up(static_cast<size_t>(pl.tiles) * 4, 256);
+  off += w.counters_bytes;
+  w.partials_off = off;
+  w.partials_bytes = static_cast<size_t>(pl.grid) * 2 * pl.npad * kTileRows * 4;
+  off += w.partials_bytes;
+  w.xg_off = off;
+  w.xg_bytes = h->perm ? round_up(static_cast<size_t>(M * h->K), 256) : 0;
+  off += w.xg_bytes;
+  w.total_device = off;
+  w.stage_x_off = off;
+  off += round_up(static_cast<size_t>(M * h->K), 256);
+  w.stage_sx_off = off;
+  off += round_up(static_cast<size_t>(M) * 4, 256);
+  w.stage_y_off = off;
+  off += round_up(static_cast<size_t>(M * h->N) * 2, 256);
+  w.total_host = off;
+  return pl;
+}
+
+spense_status check_gemm_args(const spense_packed* Wp, int64_t M, void* workspace, int* dev,
+                              DeviceInfo* info) {
+  if (Wp == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
+  if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
+  if (workspace == nullptr) return fail(SPENSE_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(SPENSE_ERR_ALIGN, "workspace is not 256-byte aligned");
+  spense_status st = current_device(dev, info);
+  if (st != SPENSE_OK) return st;
+  if (*dev != Wp->device)
+    return fail(SPENSE_ERR_ARG, "handle was packed on device %d, current device is %d", Wp->device, *dev);
+  return SPENSE_OK;
+}
+
+// Enqueue the GEMM on device buffers (arguments already validated).
+spense_status run_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale, int64_t M,
+                       uint16_t* Y, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream) {
+  const uint8_t* xsrc = X;
+  if (Wp->perm != nullptr) {
+    uint8_t* xg = ws + pl.ws.xg_off;
+    cudaError_t e = launch_gather(X, Wp->perm, M, Wp->K, xg, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+    xsrc = xg;
+  }
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+  if (encode == nullptr) return fail(SPENSE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Wp->K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Wp->K)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(pl.npad)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(xsrc), dims, strides,
+                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SPENSE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+
+  GemmParams p{};
+  p.vs_t = Wp->vs_t;
+  p.e_t = Wp->e_t;
+  p.wd_t = Wp->wd_t;
+  p.s_w = Wp->s_w;
+  p.s_x = x_scale;
+  p.y = Y;
+  p.partials = reinterpret_cast<float*>(ws + pl.ws.partials_off);
+  p.counters = reinterpret_cast<unsigned int*>(ws + pl.ws.counters_off);
+  p.status = reinterpret_cast<unsigned int*>(ws);
+  p.N = static_cast<int>(Wp->N);
+  p.M = static_cast<int>(M);
+  p.Ks = static_cast<int>(Wp->Ks);
+  p.Kd = static_cast<int>(Wp->Kd);
+  p.n_tiles = pl.n_tiles;
+  p.m_tiles = pl.m_tiles;
+  p.nsb = pl.nsb;
+  p.ndb = pl.ndb;
+  p.npad = pl.npad;
+  p.grid = pl.grid;
+  p.stages = pl.stages;
+  p.nacc = pl.nacc;
+  p.tile_cost = pl.tile_cost;
+  p.total_cost = pl.total_cost;
+  p.stage_bytes = pl.stage_bytes;
+  p.b_bytes = pl.b_bytes;
+  p.tmem_cols = pl.tmem_cols;
+  cudaError_t e = launch_gemm(map, p, pl.smem_bytes, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return SPENSE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spense_last_error(void) { return g_last_error.c_str(); }
+
+const char* spense_version(void) { return "0.1.0"; }
+
+spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int64_t K,
+                          const uint8_t* mask, const int32_t* dense_idx, int64_t Kd, uint32_t flags,
+                          void* stream_v, spense_packed** out) {
+  if (out == nullptr) return fail(SPENSE_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (W == nullptr || w_scale == nullptr) return fail(SPENSE_ERR_ARG, "W or w_scale is NULL");
+  if (flags & ~SPENSE_PACK_KEEP_CANONICAL) return fail(SPENSE_ERR_ARG, "unknown flags 0x%x", flags);
+  if (N < 1 || N > (1 << 20)) return fail(SPENSE_ERR_SHAPE, "N = %lld outside [1, 2^20]", (long long)N);
+  if (K < 16 || K > (1 << 20) || K % 16 != 0)
+    return fail(SPENSE_ERR_SHAPE, "K = %lld must be a multiple of 16 in [16, 2^20]", (long long)K);
+  if (Kd < 0 || Kd > K || Kd % 16 != 0)
+    return fail(SPENSE_ERR_SHAPE, "Kd = %lld must be a multiple of 16 in [0, K]", (long long)Kd);
+  if (!aligned(W, 16) || (mask != nullptr && !aligned(mask, 16)) || !aligned(w_scale, 4))
+    return fail(SPENSE_ERR_ALIGN, "W and mask must be 16-byte aligned, w_scale 4-byte aligned");
+  if (dense_idx != nullptr) {
+    for (int64_t j = 0; j < Kd; ++j) {
+      if (dense_idx[j] < 0 || dense_idx[j] >= K)
+        return fail(SPENSE_ERR_DENSE_IDX, "dense_idx[%lld] = %d outside [0, K)", (long long)j, dense_idx[j]);
+      if (j > 0 && dense_idx[j] <= dense_idx[j - 1])
+        return fail(SPENSE_ERR_DENSE_IDX, "dense_idx is not strictly ascending at %lld", (long long)j);
+    }
+  }
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+
+  spense_packed* h = new (std::nothrow) spense_packed();
+  if (h == nullptr) return fail(SPENSE_ERR_OOM, "host allocation failed");
+  h->device = dev;
+  h->N = N;
+  h->K = K;
+  h->Kd = Kd;
+  h->Ks = K - Kd;
+  h->n_tiles = static_cast<int>((N + kTileRows - 1) / kTileRows);
+  h->nsb = static_cast<int>((h->Ks + kSparseBlockCols - 1) / kSparseBlockCols);
+  h->ndb = static_cast<int>((Kd + kDenseBlockCols - 1) / kDenseBlockCols);
+  const bool keep_canon = (flags & SPENSE_PACK_KEEP_CANONICAL) != 0;
+
+  auto alloc = [&](void** p, size_t bytes) -> cudaError_t {
+    if (bytes == 0) return cudaSuccess;
+    return cudaMalloc(p, bytes);
+  };
+  cudaError_t e = cudaSuccess;
+  const size_t nt = static_cast<size_t>(h->n_tiles);
+  if (e == cudaSuccess) e = alloc(reinterpret_cast<void**>(&h->vs_t), nt * h->nsb * kBlockBytes);
+  if (e == cudaSuccess) e = alloc(reinterpret_cast<void**>(&h->e_t), nt * h->nsb * kMetaBlockBytes);
+  if (e == cudaSuccess) e = alloc(reinterpret_cast<void**>(&h->wd_t), nt * h->ndb * kBlockBytes);
+  if (e == cudaSuccess) e = alloc(reinterpret_cast<void**>(&h->s_w), static_cast<size_t>(N) * 4);
+  if (e == cudaSuccess && dense_idx != nullptr)
+    e = alloc(reinterpret_cast<void**>(&h->perm), static_cast<size_t>(K) * 4);
+  if (e == cudaSuccess && keep_canon) {
+    e = alloc(reinterpret_cast<void**>(&h->vs_c), static_cast<size_t>(N * (h->Ks / 2)));
+    if (e == cudaSuccess) e = alloc(reinterpret_cast<void**>(&h->e_c), static_cast<size_t>(N * (h->Ks / 8)));
+    if (e == cudaSuccess) e = alloc(reinterpret_cast<void**>(&h->wd_c), static_cast<size_t>(N * Kd));
+  }
+  unsigned int* err_d = nullptr;
+  if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&err_d), sizeof(unsigned int));
+  if (e != cudaSuccess) {
+    free_handle(h);
+    if (err_d) cudaFree(err_d);
+    return cuda_fail(e, "pack allocation");
+  }
+  if (dense_idx != nullptr) {
+    std::vector<int32_t> perm;
+    perm.reserve(static_cast<size_t>(K));
+    std::vector<char> dense(static_cast<size_t>(K), 0);
+    for (int64_t j = 0; j < Kd; ++j) dense[static_cast<size_t>(dense_idx[j])] = 1;
+    for (int64_t k = 0; k < K; ++k)
+      if (!dense[static_cast<size_t>(k)]) perm.push_back(static_cast<int32_t>(k));
+    for (int64_t j = 0; j < Kd; ++j) perm.push_back(dense_idx[j]);
+    e = cudaMemcpyAsync(h->perm, perm.data(), perm.size() * 4, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // `perm` is a host temporary
+  }
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_d, 0, sizeof(unsigned int), stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(h->s_w, w_scale, static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, stream);
+  if (e == cudaSuccess)
+    e = launch_pack(W, mask, h->perm, N, K, Kd, h->vs_t, h->e_t, h->wd_t, h->vs_c, h->e_c, h->wd_c, err_d,
+                    stream);
+  unsigned int err_h = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&err_h, err_d, sizeof(unsigned int), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  cudaFree(err_d);
+  if (e != cudaSuccess) {
+    free_handle(h);
+    return cuda_fail(e, "pack");
+  }
+  if (err_h & kPackErrNaN) {
+    free_handle(h);
+    return fail(SPENSE_ERR_NONFINITE, "W holds an e4m3 NaN byte");
+  }
+  if (err_h & kPackErrMask) {
+    free_handle(h);
+    return fail(SPENSE_ERR_MASK, "a group of four in the mask keeps more than two entries");
+  }
+  *out = h;
+  return ok();
+}
+
+spense_status spense_free(spense_packed* Wp) {
+  free_handle(Wp);
+  return ok();
+}
+
+size_t spense_gemm_workspace_size(const spense_packed* Wp, int64_t M) {
+  if (Wp == nullptr || M < 1 || M > 65535) return 0;
+  int dev = 0;
+  DeviceInfo info;
+  if (current_device(&dev, &info) != SPENSE_OK) return 0;
+  return make_plan(Wp, M, info.sms).ws.total_device;
+}
+
+size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M) {
+  if (Wp == nullptr || M < 1 || M > 65535) return 0;
+  int dev = 0;
+  DeviceInfo info;
+  if (current_device(&dev, &info) != SPENSE_OK) return 0;
+  return make_plan(Wp, M, info.sms).ws.total_host;
+}
+
+spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale, int64_t M,
+                          uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream_v) {
+  if (X == nullptr || x_scale == nullptr || Y == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(x_scale, 4))
+    return fail(SPENSE_ERR_ALIGN, "X and Y must be 16-byte aligned, x_scale 4-byte aligned");
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = check_gemm_args(Wp, M, workspace, &dev, &info);
+  if (st != SPENSE_OK) return st;
+  const GemmPlan pl = make_plan(Wp, M, info.sms);
+  if (workspace_bytes < pl.ws.total_device)
+    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                pl.ws.total_device);
+  st = run_gemm(Wp, X, x_scale, M, Y, static_cast<uint8_t*>(workspace), pl,
+                static_cast<cudaStream_t>(stream_v));
+  return st == SPENSE_OK ? ok() : st;
+}
+
+spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host, const float* x_scale_host,
+                               int64_t M, uint16_t* Y_host, void* workspace, size_t workspace_bytes,
+                               void* stream_v) {
+  if (X_host == nullptr || x_scale_host == nullptr || Y_host == nullptr)
+    return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = check_gemm_args(Wp, M, workspace, &dev, &info);
+  if (st != SPENSE_OK) return st;
+  const GemmPlan pl = make_plan(Wp, M, info.sms);
+  if (workspace_bytes < pl.ws.total_host)
+    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                pl.ws.total_host);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* xd = ws + pl.ws.stage_x_off;
+  float* sxd = reinterpret_cast<float*>(ws + pl.ws.stage_sx_off);
+  uint16_t* yd = reinterpret_cast<uint16_t*>(ws + pl.ws.stage_y_off);
+  cudaError_t e = cudaMemcpyAsync(xd, X_host, static_cast<size_t>(M * Wp->K), cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(sxd, x_scale_host, static_cast<size_t>(M) * 4, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+  st = run_gemm(Wp, xd, sxd, M, yd, ws, pl, stream);
+  if (st != SPENSE_OK) return st;
+  e = cudaMemcpyAsync(Y_host, yd, static_cast<size_t>(M * Wp->N) * 2, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  return ok();
+}
+
+spense_status spense_get_info(const spense_packed* Wp, spense_packed_info* info) {
+  if (Wp == nullptr || info == nullptr) return fail(SPENSE_ERR_ARG, "NULL argument");
+  info->N = Wp->N;
+  info->K = Wp->K;
+  info->Ks = Wp->Ks;
+  info->Kd = Wp->Kd;
+  info->n_tiles = Wp->n_tiles;
+  info->sparse_blocks = Wp->nsb;
+  info->dense_blocks = Wp->ndb;
+  info->Vs_t = Wp->vs_t;
+  info->E_t = Wp->e_t;
+  info->Wd_t = Wp->wd_t;
+  info->w_scale = Wp->s_w;
+  info->Vs = Wp->vs_c;
+  info->E = Wp->e_c;
+  info->Wd = Wp->wd_c;
+  info->perm = Wp->perm;
+  info->weight_bytes = static_cast<uint64_t>(Wp->n_tiles) *
+                       (static_cast<uint64_t>(Wp->nsb) * (kBlockBytes + kMetaBlockBytes) +
+                        static_cast<uint64_t>(Wp->ndb) * kBlockBytes);
+  return ok();
+}
+
+spense_status spense_workspace_status(void* workspace, void* stream_v, uint32_t* status_out) {
+  if (workspace == nullptr || status_out == nullptr) return fail(SPENSE_ERR_ARG, "NULL argument");
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  uint32_t word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, workspace, 4, cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess && word != 0) {
+    e = cudaMemsetAsync(workspace, 0, 4, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  }
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  *status_out = word;
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,86 @@
+// Internal declarations shared by the host ABI and the kernels of the Spense
+// library. Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "spense.h"
+
+namespace spense {
+
+constexpr int kTileRows = 128;          // weight rows per tile (MMA M)
+constexpr int kSparseBlockCols = 256;   // compacted sparse columns per block
+constexpr int kDenseBlockCols = 128;    // dense columns per block
+constexpr int kBlockBytes = 16384;      // 128 rows x 128 bytes (values or dense weights)
+constexpr int kMetaBlockBytes = 4096;   // 2 halves x 128 rows x 16 bytes
+constexpr int kMaxTokenTile = 256;      // tokens per tile (MMA N upper bound)
+constexpr int kCostSparse = 5;          // HBM bytes of a sparse block in 4 KiB units (16 + 4 KiB)
+constexpr int kCostDense = 4;           // ... of a dense block (16 KiB)
+constexpr int kGemmThreads = 192;       // warp 0 loads, warp 1 issues MMAs, warps 2-5 epilogue
+constexpr int kMaxStages = 12;
+
+// Workspace layout: [header 256 B][counters][partials][gathered X][host staging]
+struct WorkspaceLayout {
+  size_t counters_off, counters_bytes;
+  size_t partials_off, partials_bytes;
+  size_t xg_off, xg_bytes;
+  size_t stage_x_off, stage_sx_off, stage_y_off;
+  size_t total_device;  // bytes for spense_gemm
+  size_t total_host;    // bytes for spense_gemm_host
+};
+
+struct GemmPlan {
+  int npad;        // MMA N (tokens per tile, multiple of 16)
+  int m_tiles;
+  int n_tiles;
+  int tiles;       // n_tiles * m_tiles
+  int nsb, ndb;    // sparse / dense blocks per tile
+  int tile_cost;   // kCostSparse * nsb + kCostDense * ndb
+  long long total_cost;
+  int grid;        // CTAs
+  int stages;
+  uint32_t stage_bytes;
+  uint32_t b_bytes;  // bytes of the activation region of a stage
+  int nacc;          // accumulator buffers in tensor memory
+  uint32_t tmem_cols;
+  uint32_t smem_bytes;
+  WorkspaceLayout ws;
+};
+
+struct GemmParams {
+  const uint8_t* vs_t;
+  const uint8_t* e_t;
+  const uint8_t* wd_t;
+  const float* s_w;
+  const float* s_x;
+  uint16_t* y;
+  float* partials;
+  unsigned int* counters;
+  unsigned int* status;
+  int N, M, Ks, Kd;
+  int n_tiles, m_tiles, nsb, ndb;
+  int npad, grid, stages, nacc;
+  int tile_cost;
+  long long total_cost;
+  uint32_t stage_bytes, b_bytes;
+  uint32_t tmem_cols;
+};
+
+// Kernels (defined in the .cu files).
+cudaError_t launch_pack(const uint8_t* W, const uint8_t* mask, const int32_t* perm, int64_t N,
+                        int64_t K, int64_t Kd, uint8_t* vs_t, uint8_t* e_t, uint8_t* wd_t,
+                        uint8_t* vs_c, uint8_t* e_c, uint8_t* wd_c, unsigned int* err,
+                        cudaStream_t stream);
+cudaError_t launch_gather(const uint8_t* X, const int32_t* perm, int64_t M, int64_t K, uint8_t* Xg,
+                          cudaStream_t stream);
+cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t smem_bytes,
+                        cudaStream_t stream);
+uint32_t gemm_max_smem();
+
+// Device error bits written by the pack kernel.
+constexpr unsigned int kPackErrMask = 1u;
+constexpr unsigned int kPackErrNaN = 2u;
+
+}  // namespace spense

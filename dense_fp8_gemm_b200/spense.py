@@ -1,0 +1,256 @@
+"""Python binding of the Spense C ABI (include/spense.h): argument marshalling
+only. Every step of the GEMM path runs in the CUDA library ``libspense.so``;
+there is no CPU or PyTorch fallback — if the library cannot be loaded or no
+sm_100 device is present, calls raise.
+
+PyTorch supplies device memory and streams; tensors are passed by address.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+from .build import LIB_PATH
+
+SPENSE_OK = 0
+STATUS_NAMES = {
+    0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_MASK", 5: "ERR_DENSE_IDX",
+    6: "ERR_NONFINITE", 7: "ERR_WORKSPACE", 8: "ERR_OOM", 9: "ERR_CUDA", 10: "ERR_TIMEOUT",
+    11: "ERR_UNSUPPORTED",
+}
+PACK_KEEP_CANONICAL = 1
+
+# Exported symbols, in header order.
+SYMBOLS = (
+    "spense_pack", "spense_gemm", "spense_gemm_workspace_size", "spense_gemm_host",
+    "spense_gemm_host_workspace_size", "spense_free", "spense_get_info",
+    "spense_workspace_status", "spense_last_error", "spense_version",
+)
+
+
+class SpenseError(RuntimeError):
+    def __init__(self, code: int, where: str, msg: str):
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} ({msg})")
+        self.code = code
+
+
+class PackedInfo(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("Ks", ctypes.c_int64), ("Kd", ctypes.c_int64),
+        ("n_tiles", ctypes.c_int64), ("sparse_blocks", ctypes.c_int64), ("dense_blocks", ctypes.c_int64),
+        ("Vs_t", ctypes.c_void_p), ("E_t", ctypes.c_void_p), ("Wd_t", ctypes.c_void_p),
+        ("w_scale", ctypes.c_void_p), ("Vs", ctypes.c_void_p), ("E", ctypes.c_void_p),
+        ("Wd", ctypes.c_void_p), ("perm", ctypes.c_void_p), ("weight_bytes", ctypes.c_uint64),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libspense.so (built in-tree by dense_fp8_gemm_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libspense.so not found at {LIB_PATH}; run dense_fp8_gemm_b200.build.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, SZ, U32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint32
+    L.spense_pack.argtypes = [P, P, I64, I64, P, P, I64, U32, P, ctypes.POINTER(P)]
+    L.spense_gemm.argtypes = [P, P, P, I64, P, P, SZ, P]
+    L.spense_gemm_workspace_size.argtypes = [P, I64]
+    L.spense_gemm_workspace_size.restype = SZ
+    L.spense_gemm_host.argtypes = [P, P, P, I64, P, P, SZ, P]
+    L.spense_gemm_host_workspace_size.argtypes = [P, I64]
+    L.spense_gemm_host_workspace_size.restype = SZ
+    L.spense_free.argtypes = [P]
+    L.spense_get_info.argtypes = [P, ctypes.POINTER(PackedInfo)]
+    L.spense_workspace_status.argtypes = [P, P, ctypes.POINTER(U32)]
+    L.spense_last_error.restype = ctypes.c_char_p
+    L.spense_version.restype = ctypes.c_char_p
+    for name in ("spense_pack", "spense_gemm", "spense_gemm_host", "spense_free", "spense_get_info",
+                 "spense_workspace_status"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(code: int, where: str):
+    if code != SPENSE_OK:
+        raise SpenseError(code, where, lib().spense_last_error().decode())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev_ptr(t: torch.Tensor | None, dtype, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class _DevView:
+    """Zero-copy view of library-owned device memory for torch.as_tensor."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"data": (ptr, True), "shape": tuple(shape), "typestr": typestr,
+                                         "version": 3, "strides": None}
+
+
+class PackedWeight:
+    """A packed Spense weight (owns its device buffers through the C handle)."""
+
+    def __init__(self, handle: ctypes.c_void_p):
+        self._h = handle
+        info = PackedInfo()
+        _check(lib().spense_get_info(self._h, ctypes.byref(info)), "spense_get_info")
+        self.info = info
+
+    @property
+    def handle(self):
+        return self._h
+
+    @property
+    def N(self):
+        return self.info.N
+
+    @property
+    def K(self):
+        return self.info.K
+
+    @property
+    def Ks(self):
+        return self.info.Ks
+
+    @property
+    def Kd(self):
+        return self.info.Kd
+
+    @property
+    def weight_bytes(self):
+        return int(self.info.weight_bytes)
+
+    def view(self, name: str) -> torch.Tensor | None:
+        """Read-only view of a packed array ('Vs_t', 'E_t', 'Wd_t', 'Vs', 'E', 'Wd', 'perm', 'w_scale')."""
+        i = self.info
+        nt, nsb, ndb = i.n_tiles, i.sparse_blocks, i.dense_blocks
+        shapes = {
+            "Vs_t": ((nt * nsb * 16384,), "|u1"), "E_t": ((nt * nsb * 4096,), "|u1"),
+            "Wd_t": ((nt * ndb * 16384,), "|u1"), "Vs": ((i.N, i.Ks // 2), "|u1"),
+            "E": ((i.N, i.Ks // 8), "|u1"), "Wd": ((i.N, i.Kd), "|u1"), "perm": ((i.K,), "<i4"),
+            "w_scale": ((i.N,), "<f4"),
+        }
+        shape, ts = shapes[name]
+        ptr = getattr(i, name)
+        if not ptr or int(np.prod(shape)) == 0:
+            return None
+        return torch.as_tensor(_DevView(ptr, shape, ts), device="cuda")
+
+    def free(self):
+        if self._h is not None and self._h.value:
+            _check(lib().spense_free(self._h), "spense_free")
+        self._h = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def pack(W: torch.Tensor, w_scale: torch.Tensor, Kd: int | None = None, mask: torch.Tensor | None = None,
+         dense_idx=None, keep_canonical: bool = False, stream=None) -> PackedWeight:
+    """spense_pack. W: uint8 [N, K] (e4m3 bytes) on the GPU; w_scale fp32 [N];
+    dense_idx: host int32 index list (SpenseGPT+) or None (tail of Kd columns)."""
+    N, K = W.shape
+    idx = None
+    if dense_idx is not None:
+        idx = np.ascontiguousarray(np.asarray(dense_idx), dtype=np.int32)
+        if Kd is not None and Kd != idx.shape[0]:
+            raise ValueError("Kd disagrees with len(dense_idx)")
+        Kd = idx.shape[0]
+    if Kd is None:
+        raise ValueError("Kd (or dense_idx) is required")
+    out = ctypes.c_void_p()
+    code = lib().spense_pack(
+        _dev_ptr(W, torch.uint8, "W"), _dev_ptr(w_scale, torch.float32, "w_scale"), N, K,
+        _dev_ptr(mask, torch.uint8, "mask"),
+        None if idx is None else idx.ctypes.data_as(ctypes.c_void_p), Kd,
+        PACK_KEEP_CANONICAL if keep_canonical else 0, _stream(stream), ctypes.byref(out))
+    _check(code, "spense_pack")
+    return PackedWeight(out)
+
+
+def workspace_size(pw: PackedWeight, M: int) -> int:
+    n = lib().spense_gemm_workspace_size(pw.handle, M)
+    if n == 0:
+        _check(1, "spense_gemm_workspace_size")
+    return int(n)
+
+
+def host_workspace_size(pw: PackedWeight, M: int) -> int:
+    n = lib().spense_gemm_host_workspace_size(pw.handle, M)
+    if n == 0:
+        _check(1, "spense_gemm_host_workspace_size")
+    return int(n)
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zero-filled workspace (the ABI requires zeros before first use)."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device or "cuda")
+
+
+def gemm(pw: PackedWeight, X: torch.Tensor, x_scale: torch.Tensor, Y: torch.Tensor | None = None,
+         workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """spense_gemm: Y [M, N] bf16 = X [M, K] e4m3 x packed W^T, scaled."""
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, pw.N), dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = new_workspace(workspace_size(pw, M), X.device)
+    code = lib().spense_gemm(pw.handle, _dev_ptr(X, torch.uint8, "X"),
+                             _dev_ptr(x_scale, torch.float32, "x_scale"), M,
+                             _dev_ptr(Y, torch.bfloat16, "Y"), _dev_ptr(workspace, torch.uint8, "workspace"),
+                             workspace.numel(), _stream(stream))
+    _check(code, "spense_gemm")
+    return Y
+
+
+def gemm_host(pw: PackedWeight, X_host: torch.Tensor, x_scale_host: torch.Tensor, Y_host: torch.Tensor,
+              workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """spense_gemm_host: host (pinned) X, x_scale in; host Y out; synchronous."""
+    for t, name in ((X_host, "X"), (x_scale_host, "x_scale"), (Y_host, "Y")):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor")
+    M = X_host.shape[0]
+    code = lib().spense_gemm_host(pw.handle, ctypes.c_void_p(X_host.data_ptr()),
+                                  ctypes.c_void_p(x_scale_host.data_ptr()), M,
+                                  ctypes.c_void_p(Y_host.data_ptr()),
+                                  _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                  _stream(stream))
+    _check(code, "spense_gemm_host")
+    return Y_host
+
+
+def workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    """Reads and clears the device status word of a workspace (0 = all good)."""
+    out = ctypes.c_uint32()
+    _check(lib().spense_workspace_status(_dev_ptr(workspace, torch.uint8, "workspace"), _stream(stream),
+                                         ctypes.byref(out)), "spense_workspace_status")
+    return int(out.value)
+
+
+def version() -> str:
+    return lib().spense_version().decode()

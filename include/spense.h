@@ -1,0 +1,196 @@
+/*
+ * spense.h — C ABI of the Spense hybrid 2:4-sparse + dense FP8 weight GEMM for
+ * NVIDIA B200 (sm_100a).
+ *
+ *   Y[m][n] = bf16( s_x[m] * s_w[n] * sum_k X[m][k] * Wm[n][k] )
+ *
+ * where Wm is the weight matrix W [N x K] (FP8 e4m3) after its sparse region
+ * has been pruned to 2:4. The operation is the one stated on the page
+ * "SpenseGPT: Practical One-shot Pruning Enabling Sparse and Dense GEMMs for
+ * LLM Inference" (gist.science technical summary):
+ *   - Technical Summary §1 (Problem Statement): 2:4 semi-structured sparsity,
+ *     two of every four consecutive weights are zero;
+ *   - §2.A (The Spense Format): W is split along its input dimension into a
+ *     contiguous 2:4 region and a contiguous dense region; the input-split
+ *     execution runs the sparse GEMM on the first part of the input and the
+ *     dense GEMM on the second part and accumulates both. Here both parts are
+ *     contracted into one fp32 accumulator by one kernel;
+ *   - §2.B (Dense Index Selection Strategies): SpenseGPT keeps the last p% of
+ *     the input indices dense (dense_idx == NULL); SpenseGPT+ keeps an
+ *     arbitrary score-selected set dense and permutes it into one contiguous
+ *     block, which leaves Y unchanged (dense_idx != NULL);
+ *   - §4 (Experimental Results): FP8 precision on B200.
+ * The FP8 format (OCP e4m3fn), the fp32 per-output-channel and per-token
+ * scales and the bf16 output are this library's reading of "FP8 precision".
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA device addresses on the current device; host
+ *     pointers are plain host memory. Nothing is retained after a call returns
+ *     except by spense_pack, which copies what it needs into the handle.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   - Errors are returned as spense_status codes; nothing aborts or throws. On
+ *     failure outputs are left untouched and *out handles are set to NULL.
+ *     spense_last_error() gives a message for the calling thread.
+ *   - Requires a compute capability 10.x device (B200); otherwise
+ *     SPENSE_ERR_UNSUPPORTED.
+ */
+#ifndef SPENSE_H_
+#define SPENSE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPENSE_API __attribute__((visibility("default")))
+#else
+#define SPENSE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum spense_status {
+  SPENSE_OK = 0,
+  SPENSE_ERR_ARG = 1,          /* NULL pointer, unknown flag, or bad argument */
+  SPENSE_ERR_SHAPE = 2,        /* shape outside the supported set (see below) */
+  SPENSE_ERR_ALIGN = 3,        /* a device pointer is not 16-byte aligned */
+  SPENSE_ERR_MASK = 4,         /* a group of four in the mask keeps more than two */
+  SPENSE_ERR_DENSE_IDX = 5,    /* dense_idx not strictly ascending or out of [0, K) */
+  SPENSE_ERR_NONFINITE = 6,    /* W holds an e4m3 NaN byte (0x7F or 0xFF) */
+  SPENSE_ERR_WORKSPACE = 7,    /* workspace NULL or smaller than required */
+  SPENSE_ERR_OOM = 8,          /* device allocation failed */
+  SPENSE_ERR_CUDA = 9,         /* a CUDA runtime call failed */
+  SPENSE_ERR_TIMEOUT = 10,     /* a kernel gave up waiting (reported via the status word) */
+  SPENSE_ERR_UNSUPPORTED = 11  /* no compute capability 10.x device */
+} spense_status;
+
+/* Opaque packed weight. Owns its device buffers. */
+typedef struct spense_packed spense_packed;
+
+/* spense_pack flags */
+#define SPENSE_PACK_KEEP_CANONICAL 1u /* also keep the untiled Vs / E / Wd arrays (for inspection) */
+
+/*
+ * spense_pack — split W into its 2:4 region and dense region and store both in
+ * the layout the GEMM kernel streams (Technical Summary §2.A, §2.B).
+ *
+ *   W         device, e4m3 bytes [N][K] row-major (K contiguous). Read only.
+ *   w_scale   device, fp32 [N], per-output-channel scale s_w. Copied.
+ *   N, K      1 <= N <= 2^20, 16 <= K <= 2^20, K % 16 == 0.
+ *   mask      device, bytes [N][K] row-major, nonzero = keep, read on the sparse
+ *             columns only; or NULL to keep the two largest magnitudes of every
+ *             group of four (ties to the lower index).
+ *   dense_idx HOST, int32 [Kd] strictly ascending in [0, K): the dense columns
+ *             (SpenseGPT+); or NULL for the last Kd columns (SpenseGPT).
+ *   Kd        number of dense columns, 0 <= Kd <= K, Kd % 16 == 0.
+ *   flags     0 or SPENSE_PACK_KEEP_CANONICAL.
+ *   out       receives the handle.
+ *
+ * Sparse region: the Ks = K - Kd non-dense columns in ascending order, grouped
+ * four by four. A group keeps the mask's entries, or its top two; a mask group
+ * keeping fewer than two is padded with its lowest unkept index (stored value
+ * 0). More than two kept -> SPENSE_ERR_MASK.
+ *
+ * Stored format (the "tiled" arrays; rows padded to a multiple of 128, padding
+ * values 0, padding metadata 0x44):
+ *   Vs_t [ceil(N/128)][ceil(Ks/256)][128 rows][128 B]  kept values, two per
+ *        group in index order; byte c of row r at r*128 + ((c/16)^(r%8))*16 + c%16.
+ *   E_t  [ceil(N/128)][ceil(Ks/256)][2][128 rows][16 B]  2-bit index pairs,
+ *        one nibble per group (i0 | i1 << 2), group 2j in the low nibble of
+ *        byte j; half h holds the row's metadata bytes [16h, 16h+16) of the block.
+ *   Wd_t [ceil(N/128)][ceil(Kd/128)][128 rows][128 B]  dense columns in
+ *        dense_idx order, swizzled like Vs_t.
+ * With SPENSE_PACK_KEEP_CANONICAL the untiled Vs [N][Ks/2], E [N][Ks/8] and
+ * Wd [N][Kd] are kept as well.
+ *
+ * Synchronizes `stream` (mask and NaN errors are found on the device).
+ * Errors: ARG, SHAPE, ALIGN (W, mask), MASK, DENSE_IDX, NONFINITE, OOM, CUDA,
+ * UNSUPPORTED.
+ */
+SPENSE_API spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int64_t K,
+                          const uint8_t* mask, const int32_t* dense_idx, int64_t Kd,
+                          uint32_t flags, void* stream, spense_packed** out);
+
+/*
+ * spense_gemm — Y = X * Wm^T with scales (Technical Summary §2.A input-split,
+ * both regions into one fp32 accumulator; §2.B the activations are gathered
+ * into the packed column order when dense_idx was given).
+ *
+ *   Wp         packed weight from spense_pack.
+ *   X          device, e4m3 bytes [M][K] row-major, 16-byte aligned.
+ *   x_scale    device, fp32 [M], per-token scale s_x.
+ *   M          1 <= M <= 65535.
+ *   Y          device, bf16 [M][N] row-major (round to nearest even), 16-byte aligned.
+ *   workspace  device scratch of at least spense_gemm_workspace_size(Wp, M)
+ *              bytes, 256-byte aligned, ZERO-FILLED before its first use. Every
+ *              completed call leaves its counter region zero again, so one
+ *              workspace can serve any number of calls issued in stream order
+ *              (not concurrently). After SPENSE_ERR_TIMEOUT, zero it again.
+ *
+ * Asynchronous on `stream`. Device-side failures (a wait that gave up) are
+ * recorded in the workspace's status word: see spense_workspace_status.
+ * Errors: ARG, SHAPE, ALIGN, WORKSPACE, CUDA, UNSUPPORTED.
+ */
+SPENSE_API spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale,
+                          int64_t M, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
+/* Bytes of workspace spense_gemm needs for this handle and token count; 0 on a
+ * bad argument. */
+SPENSE_API size_t spense_gemm_workspace_size(const spense_packed* Wp, int64_t M);
+
+/*
+ * spense_gemm_host — the same GEMM on HOST buffers: copies X [M][K] and
+ * x_scale [M] from host memory into the workspace, runs spense_gemm, copies Y
+ * [M][N] back to host memory and synchronizes `stream` before returning.
+ * Host buffers should be pinned for asynchronous copies. workspace must hold
+ * spense_gemm_host_workspace_size(Wp, M) bytes (zero-filled before first use).
+ */
+SPENSE_API spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host,
+                               const float* x_scale_host, int64_t M, uint16_t* Y_host,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+SPENSE_API size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M);
+
+/* Releases the handle and its device buffers (stream-ordered on the stream the
+ * handle was packed on). NULL is accepted. */
+SPENSE_API spense_status spense_free(spense_packed* Wp);
+
+/* Shapes and device addresses of a packed weight (for inspection and tests).
+ * Canonical pointers are NULL unless packed with SPENSE_PACK_KEEP_CANONICAL. */
+typedef struct spense_packed_info {
+  int64_t N, K, Ks, Kd;
+  int64_t n_tiles, sparse_blocks, dense_blocks;
+  const void* Vs_t;       /* n_tiles * sparse_blocks * 16384 bytes */
+  const void* E_t;        /* n_tiles * sparse_blocks * 4096 bytes */
+  const void* Wd_t;       /* n_tiles * dense_blocks * 16384 bytes */
+  const void* w_scale;    /* fp32 [N] */
+  const void* Vs;         /* [N][Ks/2] or NULL */
+  const void* E;          /* [N][Ks/8] or NULL */
+  const void* Wd;         /* [N][Kd] or NULL */
+  const int32_t* perm;    /* device int32 [K]: sparse columns then dense columns, or NULL (tail) */
+  uint64_t weight_bytes;  /* bytes of Vs_t + E_t + Wd_t */
+} spense_packed_info;
+
+SPENSE_API spense_status spense_get_info(const spense_packed* Wp, spense_packed_info* info);
+
+/* Reads and clears the status word a workspace carries. *status_out receives 0
+ * when every kernel that used the workspace completed normally, else a bitwise
+ * OR of SPENSE_DEVICE_* codes. Synchronizes `stream`. */
+#define SPENSE_DEVICE_TIMEOUT_PRODUCER 0x1u
+#define SPENSE_DEVICE_TIMEOUT_MMA 0x2u
+#define SPENSE_DEVICE_TIMEOUT_EPILOGUE 0x4u
+SPENSE_API spense_status spense_workspace_status(void* workspace, void* stream, uint32_t* status_out);
+
+/* Message describing the last error on the calling thread ("" if none). */
+SPENSE_API const char* spense_last_error(void);
+
+/* Library version, "major.minor.patch". */
+SPENSE_API const char* spense_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPENSE_H_ */

@@ -1,0 +1,118 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+include/spense.h declares, and rejects bad arguments with status codes before
+touching a device. No GPU is needed."""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import dense_fp8_gemm_b200.build as build_mod
+from dense_fp8_gemm_b200 import spense
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "spense.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build_mod.build()
+    return spense.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return re.findall(r"SPENSE_API\s+[\w\s\*]*?\b(spense_\w+)\s*\(", text)
+
+
+def test_header_declares_the_binding_symbols():
+    assert sorted(declared_symbols()) == sorted(spense.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", build_mod.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(declared_symbols()) <= exported
+    # nothing else leaks out under the spense_ prefix
+    assert {s for s in exported if s.startswith("spense_")} == set(declared_symbols())
+
+
+def test_version(L):
+    assert re.fullmatch(r"\d+\.\d+\.\d+", spense.version())
+
+
+def _pack_raw(L, W=0x1000, w_scale=0x2000, N=128, K=256, mask=None, dense_idx=None, Kd=64, flags=0):
+    out = ctypes.c_void_p(0x1234)
+    code = L.spense_pack(ctypes.c_void_p(W) if W else None, ctypes.c_void_p(w_scale) if w_scale else None,
+                         N, K, ctypes.c_void_p(mask) if mask else None, dense_idx, Kd, flags, None,
+                         ctypes.byref(out))
+    return code, out
+
+
+def test_pack_rejects_null_and_flags(L):
+    code, out = _pack_raw(L, W=0)
+    assert code == 1 and out.value is None
+    assert b"NULL" in L.spense_last_error()
+    code, _ = _pack_raw(L, flags=0x10)
+    assert code == 1
+    code = L.spense_pack(ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 128, 256, None, None, 64, 0, None,
+                         None)
+    assert code == 1
+
+
+@pytest.mark.parametrize("N,K,Kd", [(0, 256, 64), (128, 8, 0), (128, 250, 64), (128, 256, 72),
+                                    (128, 256, 272), (128, 256, -16), (1 << 21, 256, 0)])
+def test_pack_rejects_shapes(L, N, K, Kd):
+    code, _ = _pack_raw(L, N=N, K=K, Kd=Kd)
+    assert code == 2, L.spense_last_error()
+
+
+def test_pack_rejects_misalignment(L):
+    assert _pack_raw(L, W=0x1001)[0] == 3
+    assert _pack_raw(L, mask=0x3008)[0] == 3
+    assert _pack_raw(L, w_scale=0x2002)[0] == 3
+
+
+@pytest.mark.parametrize("idx", [[3, 2], [1, 1], [0, 256], [-1, 5]])
+def test_pack_rejects_dense_idx(L, idx):
+    arr = np.zeros(16, np.int32)
+    arr[:] = np.arange(16) * 2
+    arr[: len(idx)] = idx
+    if idx == [0, 256]:
+        arr = np.arange(16, dtype=np.int32)
+        arr[-1] = 256
+    code, _ = _pack_raw(L, dense_idx=arr.ctypes.data_as(ctypes.c_void_p), Kd=16)
+    assert code == 5, L.spense_last_error()
+
+
+def test_gemm_rejects_null(L):
+    code = L.spense_gemm(None, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 1, ctypes.c_void_p(0x3000),
+                         ctypes.c_void_p(0x4000), 1 << 20, None)
+    assert code == 1
+    code = L.spense_gemm(ctypes.c_void_p(0x10), None, ctypes.c_void_p(0x2000), 1, ctypes.c_void_p(0x3000),
+                         ctypes.c_void_p(0x4000), 1 << 20, None)
+    assert code == 1
+    code = L.spense_gemm(ctypes.c_void_p(0x10), ctypes.c_void_p(0x1008), ctypes.c_void_p(0x2000), 1,
+                         ctypes.c_void_p(0x3000), ctypes.c_void_p(0x4000), 1 << 20, None)
+    assert code == 3
+    assert L.spense_gemm_workspace_size(None, 4) == 0
+    assert L.spense_gemm_host_workspace_size(None, 4) == 0
+    assert L.spense_get_info(None, None) == 1
+    assert L.spense_free(None) == 0
+
+
+def test_valid_arguments_without_a_device_report_unsupported(L):
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if has_gpu:
+        pytest.skip("a GPU is present")
+    code, out = _pack_raw(L)
+    assert code == 11 and out.value is None

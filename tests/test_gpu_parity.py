@@ -1,0 +1,227 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Packing is compared byte for byte (tiled storage and canonical arrays); the
+GEMM output must satisfy |y - y_ref| <= 4e-3 |y_ref| + 1e-5 sum_k |w_k x_k|
+on every element the oracle computes (all of them for small cases, sampled
+rows spanning every region of the tile grid for the full-size workloads).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dense_fp8_gemm_b200 import spense, synth, workloads
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 4e-3, 1e-5
+
+
+def _dev(a, dtype=None):
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.cuda() if dtype is None else t.to(dtype).cuda()
+
+
+def _assert_close(y_gpu, yref, bound, what=""):
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    ok = oracle.within_tolerance(y, yref, bound, REL, ABS)
+    if not ok.all():
+        bad = np.argwhere(~ok)
+        i, j = bad[0]
+        raise AssertionError(
+            f"{what}: {len(bad)} of {ok.size} outside tolerance; first at {tuple(bad[0])}: "
+            f"gpu {y[i, j]!r} ref {yref[i, j]!r} bound {bound[i, j]!r}")
+
+
+def _make(seed, M, N, K, Kd, scattered=False, w_std=0.02):
+    X, s_x = synth.quantize_rows(synth.normal(seed, 1, (M, K), 1.0))
+    W, s_w = synth.quantize_rows(synth.normal(seed, 2, (N, K), w_std))
+    idx = synth.scored_dense_idx(seed, 3, K, Kd) if scattered else None
+    return X, s_x, W, s_w, idx
+
+
+def _run(pw, X, s_x):
+    Xd, sxd = _dev(X), _dev(s_x)
+    ws = spense.new_workspace(spense.workspace_size(pw, X.shape[0]))
+    Y = spense.gemm(pw, Xd, sxd, workspace=ws)
+    torch.cuda.synchronize()
+    assert spense.workspace_status(ws) == 0
+    return Y, ws
+
+
+# --------------------------------------------------------------------------- packing, bit-exact
+
+PACK_CASES = [
+    # N, K, Kd, scattered, mask
+    (256, 512, 128, False, None),          # the tiny workload
+    (200, 640, 160, False, None),          # ragged rows, ragged sparse and dense blocks
+    (130, 1024, 0, False, None),           # pure 2:4
+    (64, 512, 512, False, None),           # pure dense
+    (256, 1024, 336, True, None),          # SpenseGPT+ scattered dense set
+    (192, 768, 256, False, (0, 1, 2)),     # explicit masks with 0, 1 or 2 kept
+    (160, 896, 224, True, (1, 2)),         # masks over a scattered sparse region
+]
+
+
+@pytest.mark.parametrize("N,K,Kd,scattered,keeps", PACK_CASES)
+def test_pack_bit_exact(N, K, Kd, scattered, keeps):
+    _, _, W, s_w, idx = _make(100 + N, 1, N, K, Kd, scattered)
+    mask = None
+    if keeps is not None:
+        sparse_cols = np.setdiff1d(np.arange(K), idx) if scattered else np.arange(K - Kd)
+        mask = synth.random_mask(100 + N, 7, N, K, keeps, sparse_cols)
+    ref = oracle.pack(W, mask=mask, dense_idx=idx, Kd=Kd)
+    Ks = K - Kd
+    tref = oracle.tile(ref["Vs"], ref["E"], ref["Wd"], N, Ks, Kd)
+    pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd, mask=None if mask is None else _dev(mask), dense_idx=idx,
+                     keep_canonical=True)
+    torch.cuda.synchronize()
+    for name, key in (("Vs_t", "Vs_t"), ("E_t", "E_t"), ("Wd_t", "Wd_t")):
+        v = pw.view(name)
+        got = np.zeros(0, np.uint8) if v is None else v.cpu().numpy()
+        np.testing.assert_array_equal(got, tref[key], err_msg=name)
+    for name in ("Vs", "E", "Wd"):
+        v = pw.view(name)
+        got = np.zeros(ref[name].shape, np.uint8) if v is None else v.cpu().numpy()
+        np.testing.assert_array_equal(got, ref[name], err_msg=name)
+    np.testing.assert_array_equal(pw.view("w_scale").cpu().numpy(), s_w)
+    pw.free()
+
+
+def test_pack_rejects_bad_mask_and_nan():
+    N, K, Kd = 128, 256, 64
+    _, _, W, s_w, _ = _make(5, 1, N, K, Kd)
+    mask = np.ones((N, K), np.uint8)
+    mask[:, :K - Kd] = synth.random_mask(5, 9, N, K - Kd, (2,))
+    mask[17, 8:11] = 1  # three kept in group 2 of row 17
+    mask[17, 11] = 0
+    with pytest.raises(spense.SpenseError) as ei:
+        spense.pack(_dev(W), _dev(s_w), Kd=Kd, mask=_dev(mask))
+    assert ei.value.code == 4
+    W2 = W.copy()
+    W2[3, 200] = 0xFF
+    with pytest.raises(spense.SpenseError) as ei:
+        spense.pack(_dev(W2), _dev(s_w), Kd=Kd)
+    assert ei.value.code == 6
+
+
+# --------------------------------------------------------------------------- GEMM, all elements
+
+SMALL = [
+    # M, N, K, Kd, scattered
+    (8, 256, 512, 128, False),     # the tiny workload shape
+    (1, 384, 1024, 256, False),
+    (5, 200, 640, 160, False),     # ragged rows and blocks
+    (16, 512, 2048, 512, False),
+    (17, 256, 1024, 256, False),   # tokens just past one MMA N step
+    (40, 384, 768, 0, False),      # pure 2:4
+    (33, 256, 768, 768, False),    # pure dense
+    (24, 320, 1536, 384, True),    # SpenseGPT+ gather
+    (64, 1024, 512, 128, False),
+    (128, 256, 512, 128, False),
+    (200, 256, 512, 128, False),
+    (256, 384, 512, 128, False),
+    (300, 256, 512, 128, False),   # two token tiles
+    (600, 128, 256, 64, True),     # three token tiles with a gather
+]
+
+
+@pytest.mark.parametrize("M,N,K,Kd,scattered", SMALL)
+def test_gemm_matches_oracle(M, N, K, Kd, scattered):
+    X, s_x, W, s_w, idx = _make(M * 7 + N, M, N, K, Kd, scattered)
+    ref = oracle.pack(W, dense_idx=idx, Kd=Kd)
+    yref, bound = oracle.gemm(X, s_x, W, s_w, keep=ref["keep"])
+    pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd, dense_idx=idx)
+    Y, _ = _run(pw, X, s_x)
+    _assert_close(Y, yref, bound, f"M={M} N={N} K={K} Kd={Kd}")
+
+
+def test_gemm_with_explicit_mask():
+    M, N, K, Kd = 12, 384, 1024, 256
+    X, s_x, W, s_w, _ = _make(21, M, N, K, Kd)
+    mask = synth.random_mask(21, 8, N, K, (0, 1, 2), np.arange(K - Kd))
+    ref = oracle.pack(W, mask=mask, Kd=Kd)
+    yref, bound = oracle.gemm(X, s_x, W, s_w, keep=ref["keep"])
+    pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd, mask=_dev(mask))
+    Y, _ = _run(pw, X, s_x)
+    _assert_close(Y, yref, bound, "mask")
+
+
+def test_gemm_is_deterministic_and_host_path_agrees():
+    M, N, K, Kd = 16, 1024, 4096, 1024  # several CTAs share each tile
+    X, s_x, W, s_w, _ = _make(31, M, N, K, Kd)
+    pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd)
+    Y1, ws = _run(pw, X, s_x)
+    Y2 = spense.gemm(pw, _dev(X), _dev(s_x), workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    hws = spense.new_workspace(spense.host_workspace_size(pw, M))
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    spense.gemm_host(pw, torch.from_numpy(X).pin_memory(), torch.from_numpy(s_x).pin_memory(), Yh, hws)
+    assert torch.equal(Yh.view(torch.int16), Y1.cpu().view(torch.int16))
+
+
+def test_spenseplus_with_tail_list_equals_spensegpt():
+    M, N, K, Kd = 8, 256, 1024, 256
+    X, s_x, W, s_w, _ = _make(41, M, N, K, Kd)
+    a = spense.pack(_dev(W), _dev(s_w), Kd=Kd)
+    b = spense.pack(_dev(W), _dev(s_w), dense_idx=np.arange(K - Kd, K))
+    Ya, _ = _run(a, X, s_x)
+    Yb, _ = _run(b, X, s_x)
+    assert torch.equal(Ya.view(torch.int16), Yb.view(torch.int16))
+
+
+# --------------------------------------------------------------------------- full-size workloads, sampled rows
+
+
+def _sample_rows(N, count=96, seed=0):
+    g = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, N // 2, N - 129, N - 128, N - 1]
+    rows = np.unique(np.concatenate([np.array([r for r in fixed if 0 <= r < N]),
+                                     g.choice(N, size=min(count, N), replace=False)]))
+    return rows
+
+
+def _check_workload_shape(wl, i, batches, dense_frac=None):
+    w = workloads.make_weight(wl, i, dense_frac)
+    pw = spense.pack(_dev(w.W), _dev(w.s_w), Kd=w.Kd, dense_idx=w.dense_idx)
+    rows = _sample_rows(w.N, seed=i)
+    keep = oracle.pack(w.W[rows], dense_idx=w.dense_idx, Kd=w.Kd)["keep"]
+    for M in batches:
+        X, s_x = workloads.make_activations(wl, i, M)
+        yref, bound = oracle.gemm(X, s_x, w.W[rows], w.s_w[rows], keep=keep)
+        Y, _ = _run(pw, X, s_x)
+        _assert_close(Y[:, torch.from_numpy(rows).cuda()], yref, bound,
+                      f"{wl.name}/{w.label} M={M} df={dense_frac}")
+    pw.free()
+
+
+def test_tiny_workload_all_elements():
+    wl = workloads.TINY
+    w = workloads.make_weight(wl, 0)
+    X, s_x = workloads.make_activations(wl, 0, 8)
+    ref = oracle.pack(w.W, Kd=w.Kd)
+    yref, bound = oracle.gemm(X, s_x, w.W, w.s_w, keep=ref["keep"])
+    pw = spense.pack(_dev(w.W), _dev(w.s_w), Kd=w.Kd)
+    Y, _ = _run(pw, X, s_x)
+    _assert_close(Y, yref, bound, "tiny")
+
+
+@pytest.mark.parametrize("i", range(4))
+def test_attn32b(i):
+    _check_workload_shape(workloads.ATTN32B, i, workloads.ATTN32B.batches)
+
+
+@pytest.mark.parametrize("i", range(2))
+def test_ffn32b(i):
+    _check_workload_shape(workloads.FFN32B, i, workloads.FFN32B.batches)
+
+
+@pytest.mark.parametrize("df", workloads.SPENSE_PLUS.dense_fracs)
+def test_spensegpt_plus_sweep(df):
+    _check_workload_shape(workloads.SPENSE_PLUS, 0, workloads.SPENSE_PLUS.batches, dense_frac=df)
+
+
+@pytest.mark.parametrize("i", range(6))
+def test_chain36b_layer(i):
+    _check_workload_shape(workloads.CHAIN36B, i, workloads.CHAIN36B.batches)
