@@ -36,8 +36,8 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=400)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["spense", "reference"], default="spense")
     ap.add_argument("--tokens", type=int, default=16, help="decode tokens M")
     ap.add_argument("--layers", type=int, default=8, help="weight sets rotated between steps")
@@ -83,28 +83,39 @@ def read_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs.
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Sampling starts before the warm-up; `mark(t0, t1)` records the wall-clock
+    window of the timed region and only samples inside it are summarized (all
+    samples if the window caught none, which `in_window` reports)."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 50):
         self.gpu = gpu_index
+        self.interval = interval_ms
         self.proc = None
+        self.window = None
+        self.lines = []
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.interval)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.5)  # let the first samples arrive before the work starts
         except Exception:
             self.proc = None
         return self
 
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
+            time.sleep(2 * self.interval / 1000)
             self.proc.terminate()
             try:
                 out, _ = self.proc.communicate(timeout=5)
@@ -114,24 +125,29 @@ class ClockSampler:
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
+        import datetime
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        samples = []
+        for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                samples.append((ts, float(f[2]), float(f[3]), f[6:10]))
             except ValueError:
                 continue
-            for name, val in zip(names, f[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        inside = samples
+        in_window = False
+        if self.window is not None:
+            w = [x for x in samples if self.window[0] - 0.06 <= x[0] <= self.window[1] + 0.06]
+            if w:
+                inside, in_window = w, True
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "in_window": False}
+        reasons = sorted({n for x in inside for n, v in zip(names, x[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": reasons, "samples": len(inside), "in_window": in_window}
 
 
 # ----------------------------------------------------------------------------- CPU oracle timing
@@ -278,7 +294,7 @@ def run_spense(args):
         torch.cuda.synchronize()
         return graphs, evs
 
-    def timed(graphs, steps, warmup):
+    def timed(graphs, steps, warmup, clocks=None):
         for i in range(warmup):
             graphs[i % len(graphs)].replay()
         torch.cuda.synchronize()
@@ -287,11 +303,14 @@ def run_spense(args):
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        w0 = time.time()
         e0.record()
         for i in range(steps):
             graphs[i % len(graphs)].replay()
         e1.record()
         torch.cuda.synchronize()
+        if clocks is not None:
+            clocks.mark(w0, time.time())
         if world > 1:
             dist.barrier()
         return e0.elapsed_time(e1) / 1e3  # seconds
@@ -300,7 +319,7 @@ def run_spense(args):
     g_dn, _ = capture(layers_dn)
 
     with ClockSampler(local) as clocks:
-        t_sp = timed(g_sp, args.steps, args.warmup)
+        t_sp = timed(g_sp, args.steps, args.warmup, clocks)
     t_dn = timed(g_dn, args.steps, args.warmup)
 
     if world > 1:

@@ -32,6 +32,7 @@
 // code in the workspace status word and all roles leave their loops.
 #include <algorithm>
 #include <cstdint>
+#include <cstdlib>
 #include <cuda_bf16.h>
 
 #include "sm100_ptx.cuh"
@@ -123,6 +124,40 @@ struct UnitIter {
   }
 };
 
+// Walks blocks b0, b0+1, ... keeping (tile, block, n-tile, token-tile)
+// incrementally, so the per-block path has no integer division.
+struct BlockCursor {
+  int j, nblk, m_tile, m_tiles;
+  long long n_tile;
+  __device__ BlockCursor(long long b, int nblk_, int m_tiles_) : nblk(nblk_), m_tiles(m_tiles_) {
+    const long long t = b / nblk;
+    j = static_cast<int>(b - t * nblk);
+    n_tile = t / m_tiles;
+    m_tile = static_cast<int>(t - n_tile * m_tiles);
+  }
+  __device__ void advance() {
+    if (++j == nblk) {
+      j = 0;
+      if (++m_tile == m_tiles) {
+        m_tile = 0;
+        ++n_tile;
+      }
+    }
+  }
+};
+
+// Ring position: stage index and the parity of its current use.
+struct Ring {
+  uint32_t s = 0, ph = 0, n;
+  __device__ explicit Ring(uint32_t stages) : n(stages) {}
+  __device__ void advance() {
+    if (++s == n) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
 __device__ __forceinline__ uint16_t to_bf16_bits(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
@@ -161,6 +196,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
+  // Let the next kernel in the stream start launching: its CTAs take SMs as
+  // this grid's CTAs exit and wait (griddepcontrol.wait) before reading
+  // anything this grid writes.
+  ptx::griddep_launch_dependents();
 
   const Split split(p);
   const long long b0 = split.cta_first_block(g);
@@ -169,45 +208,54 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Blocks b0..b1-1 go through the ring in order. The weight copies of the
+    // first ring's worth are issued before waiting on the previous grid (the
+    // packed weights never depend on it), the activation tiles after.
     if (lane == 0) {
       const uint64_t pol_w = ptx::policy_evict_first();
       const uint64_t pol_x = ptx::policy_evict_last();
-      UnitIter units(b0, b1, split.nblk);
-      long long t;
-      int j0, j1;
-      uint32_t it = 0;
-      bool ok = true;
-      while (ok && units.next(t, j0, j1)) {
-        const long long n_tile = t / p.m_tiles;
-        const int y0 = static_cast<int>(t % p.m_tiles) * kMaxTokenTile;
-        for (int j = j0; j < j1; ++j, ++it) {
-          const uint32_t s = it % p.stages;
-          const uint32_t ph = (it / p.stages) & 1u;
-          if (!wait_bar(ptx::smem_addr(&bars->empty[s]), ph ^ 1u, p.status,
-                        SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const uint32_t a_s = smem_base + s * p.stage_bytes;
-          const uint32_t b_s = a_s + kBlockBytes;
-          const uint32_t e_s = b_s + p.b_bytes;
-          const uint32_t full = ptx::smem_addr(&bars->full[s]);
-          const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
-          if (j < p.nsb) {
-            const size_t blk = static_cast<size_t>(n_tile) * p.nsb + j;
-            ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * box);
-            ptx::bulk_g2s(a_s, p.vs_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
-            ptx::bulk_g2s(e_s, p.e_t + blk * kMetaBlockBytes, kMetaBlockBytes, full, pol_w);
-            ptx::tma_load_2d(b_s, &tmap_x, j * kSparseBlockCols, y0, full, pol_x);
-            ptx::tma_load_2d(b_s + box, &tmap_x, j * kSparseBlockCols + 128, y0, full, pol_x);
-          } else {
-            const int jd = j - p.nsb;
-            const size_t blk = static_cast<size_t>(n_tile) * p.ndb + jd;
-            ptx::mbar_arrive_expect_tx(full, kBlockBytes + box);
-            ptx::bulk_g2s(a_s, p.wd_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
-            ptx::tma_load_2d(b_s, &tmap_x, p.Ks + jd * kDenseBlockCols, y0, full, pol_x);
-          }
+      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
+      const long long nb = b1 - b0;
+      const int pre = static_cast<int>(nb < p.stages ? nb : p.stages);
+      auto issue_w = [&](const BlockCursor& c, uint32_t s) {
+        const uint32_t a_s = smem_base + s * p.stage_bytes;
+        const uint32_t full = ptx::smem_addr(&bars->full[s]);
+        if (c.j < p.nsb) {
+          const size_t blk = static_cast<size_t>(c.n_tile) * p.nsb + c.j;
+          ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * box);
+          ptx::bulk_g2s(a_s, p.vs_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
+          ptx::bulk_g2s(a_s + kBlockBytes + p.b_bytes, p.e_t + blk * kMetaBlockBytes, kMetaBlockBytes, full,
+                        pol_w);
+        } else {
+          const size_t blk = static_cast<size_t>(c.n_tile) * p.ndb + (c.j - p.nsb);
+          ptx::mbar_arrive_expect_tx(full, kBlockBytes + box);
+          ptx::bulk_g2s(a_s, p.wd_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
         }
+      };
+      auto issue_x = [&](const BlockCursor& c, uint32_t s) {
+        const int y0 = c.m_tile * kMaxTokenTile;
+        const uint32_t b_s = smem_base + s * p.stage_bytes + kBlockBytes;
+        const uint32_t full = ptx::smem_addr(&bars->full[s]);
+        if (c.j < p.nsb) {
+          ptx::tma_load_2d(b_s, &tmap_x, c.j * kSparseBlockCols, y0, full, pol_x);
+          ptx::tma_load_2d(b_s + box, &tmap_x, c.j * kSparseBlockCols + 128, y0, full, pol_x);
+        } else {
+          ptx::tma_load_2d(b_s, &tmap_x, p.Ks + (c.j - p.nsb) * kDenseBlockCols, y0, full, pol_x);
+        }
+      };
+      BlockCursor cw(b0, split.nblk, p.m_tiles);
+      for (int i = 0; i < pre; ++i, cw.advance()) issue_w(cw, static_cast<uint32_t>(i));
+      ptx::griddep_wait();
+      BlockCursor cx(b0, split.nblk, p.m_tiles);
+      for (int i = 0; i < pre; ++i, cx.advance()) issue_x(cx, static_cast<uint32_t>(i));
+      Ring ring(static_cast<uint32_t>(p.stages));
+      for (int i = 0; i < pre; ++i) ring.advance();
+      for (long long i = pre; i < nb; ++i, ring.advance(), cw.advance()) {
+        if (!wait_bar(ptx::smem_addr(&bars->empty[ring.s]), ring.ph ^ 1u, p.status,
+                      SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag))
+          break;
+        issue_w(cw, ring.s);
+        issue_x(cw, ring.s);
       }
     }
   } else if (warp == 1) {
@@ -219,7 +267,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       UnitIter units(b0, b1, split.nblk);
       long long t;
       int j0, j1;
-      uint32_t it = 0, u = 0, ebuf = 0;
+      uint32_t u = 0, ebuf = 0;
+      Ring ring(static_cast<uint32_t>(p.stages));
       bool ok = true;
       while (ok && units.next(t, j0, j1)) {
         const uint32_t acc = u % p.nacc;
@@ -231,9 +280,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.npad);
-        for (int j = j0; j < j1; ++j, ++it) {
-          const uint32_t s = it % p.stages;
-          const uint32_t ph = (it / p.stages) & 1u;
+        for (int j = j0; j < j1; ++j, ring.advance()) {
+          const uint32_t s = ring.s;
+          const uint32_t ph = ring.ph;
           if (!wait_bar(ptx::smem_addr(&bars->full[s]), ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
                         abort_flag)) {
             ok = false;
@@ -273,6 +322,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    ptx::griddep_wait();  // s_x, Y and the workspace may belong to the previous grid
     const int et = threadIdx.x - 64;           // 0..127
     const int quarter = warp & 3;              // tensor-memory lane quarter this warp may read
     const int row = quarter * 32 + lane;
@@ -296,53 +346,105 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const float sw = row_ok ? __ldg(p.s_w + n) : 0.0f;
       const bool whole = (j0 == 0 && j1 == split.nblk);
       const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
+      // Partials are stored [slot][row][npad] so each thread owns one contiguous row.
       float* part = nullptr;
       if (!whole)
-        part = p.partials + (static_cast<size_t>(g) * 2 + split.slot(g, t)) * p.npad * kTileRows;
+        part = p.partials + ((static_cast<size_t>(g) * 2 + split.slot(g, t)) * kTileRows + row) * p.npad;
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
         uint32_t v[16];
         ptx::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), v);
         ptx::tmem_ld_wait();
+        if (whole) {
+          if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int m = c0 + i;
-          if (m < m_valid) {
-            const float a = __uint_as_float(v[i]);
-            if (whole) {
-              if (row_ok)
+            for (int i = 0; i < 16; ++i) {
+              const int m = c0 + i;
+              if (m < m_valid)
                 p.y[static_cast<size_t>(m0 + m) * p.N + n] =
-                    to_bf16_bits(a * sw * __ldg(p.s_x + m0 + m));
-            } else {
-              part[static_cast<size_t>(m) * kTileRows + row] = a;
+                    to_bf16_bits(__uint_as_float(v[i]) * sw * __ldg(p.s_x + m0 + m));
             }
           }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(part + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (c0 + 4 * q < m_valid)
+              __stcg(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
         }
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
       ++u;
       if (!whole) {
-        __threadfence();
+        // Publish this CTA's partial: the named barrier orders the 128 threads'
+        // stores before thread 0's release-acquire ticket at GPU scope.
         ptx::named_bar_sync(1, 128);
         const int g_lo = split.owner(t, 0);
         const int g_hi = split.owner(t, split.nblk - 1);
         if (et == 0) {
-          const unsigned int old = atomicAdd(p.counters + t, 1u);
+          const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
           bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
         }
         ptx::named_bar_sync(1, 128);
         const int finisher = *reinterpret_cast<volatile int*>(&bars->fix_flag);
         if (finisher) {
-          __threadfence();
-          for (int m = 0; m < m_valid; ++m) {
-            float sum = 0.0f;
-            for (int gg = g_lo; gg <= g_hi; ++gg) {
-              const float* pp =
-                  p.partials + (static_cast<size_t>(gg) * 2 + split.slot(gg, t)) * p.npad * kTileRows;
-              sum += __ldcg(pp + static_cast<size_t>(m) * kTileRows + row);
+          // Contributors g_lo..g_hi own consecutive block ranges of tile t. Every
+          // contributor after g_lo starts inside t, so its partial is in slot 0;
+          // g_lo uses slot 1 when its range started in an earlier tile. The sum
+          // runs in contributor order.
+          const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
+          const float* lo_part =
+              p.partials + (static_cast<size_t>(g_lo) * 2 + split.slot(g_lo, t)) * slot_elems +
+              static_cast<size_t>(row) * p.npad;
+          const float* next_part =
+              p.partials + (static_cast<size_t>(g_lo + 1) * 2) * slot_elems + static_cast<size_t>(row) * p.npad;
+          const size_t stride = 2 * slot_elems;  // from contributor gg to gg + 1 (slot 0)
+          const int others = g_hi - g_lo;
+          for (int c0 = 0; c0 < m_valid; c0 += 16) {
+            const int nq = min(4, (m_valid - c0 + 3) >> 2);  // float4 groups holding valid tokens
+            float4 a[4], b[4], c[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (q < nq) a[q] = __ldcg(reinterpret_cast<const float4*>(lo_part + c0) + q);
+            int k = 0;
+            for (; k + 2 <= others; k += 2) {
+              const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
+              const float4* pc = reinterpret_cast<const float4*>(next_part + (k + 1) * stride + c0);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (q < nq) {
+                  b[q] = __ldcg(pb + q);
+                  c[q] = __ldcg(pc + q);
+                }
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (q < nq) {
+                  a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
+                  a[q].x += c[q].x; a[q].y += c[q].y; a[q].z += c[q].z; a[q].w += c[q].w;
+                }
             }
-            if (row_ok)
-              p.y[static_cast<size_t>(m0 + m) * p.N + n] = to_bf16_bits(sum * sw * __ldg(p.s_x + m0 + m));
+            if (k < others) {
+              const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                if (q < nq) {
+                  b[q] = __ldcg(pb + q);
+                  a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
+                }
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float r4[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                  const int m = c0 + 4 * q + i;
+                  if (q < nq && m < m_valid)
+                    p.y[static_cast<size_t>(m0 + m) * p.N + n] = to_bf16_bits(r4[i] * sw * __ldg(p.s_x + m0 + m));
+                }
+              }
+            }
           }
           if (et == 0) atomicExch(p.counters + t, 0u);
         }
@@ -375,8 +477,24 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
     if (st != cudaSuccess) return st;
     configured_for = dev;
   }
-  spense_gemm_kernel<<<p.grid, kGemmThreads, smem_bytes, stream>>>(tmap_x, p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: CTAs of this grid may start on SMs the
+  // previous kernel in the stream has released; they prefetch weights and then
+  // wait (griddepcontrol.wait) before reading anything that kernel may write.
+  static const bool pdl = [] {
+    const char* e = std::getenv("SPENSE_PDL");
+    return !(e != nullptr && e[0] == '0');
+  }();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned int>(p.grid));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem_bytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, spense_gemm_kernel, tmap_x, p);
 }
 
 }  // namespace spense

@@ -4,6 +4,7 @@
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <new>
@@ -109,6 +110,17 @@ void free_handle(spense_packed* h) {
   delete h;
 }
 
+// Minimum streamed weight per CTA in 4 KiB units (default 20 = four 2:4 blocks);
+// SPENSE_MIN_CTA_WEIGHT overrides it for tuning.
+long long min_cta_weight() {
+  static const long long v = [] {
+    const char* e = std::getenv("SPENSE_MIN_CTA_WEIGHT");
+    long long x = e ? std::atoll(e) : 20;
+    return x > 0 ? x : 20;
+  }();
+  return v;
+}
+
 // Launch plan for (handle, M) on a device with `sms` SMs.
 GemmPlan make_plan(const spense_packed* h, int64_t M, int sms) {
   GemmPlan pl{};
@@ -120,8 +132,10 @@ GemmPlan make_plan(const spense_packed* h, int64_t M, int sms) {
   pl.ndb = h->ndb;
   pl.tile_cost = kCostSparse * pl.nsb + kCostDense * pl.ndb;
   pl.total_cost = static_cast<long long>(pl.tiles) * pl.tile_cost;
-  // At least one maximal block of weight per CTA, so no CTA owns an empty range.
-  long long grid = pl.total_cost / kCostSparse;
+  // Each CTA gets at least min_cta_weight() units of streamed bytes (never less
+  // than one maximal block, so no CTA owns an empty range): small matrices are
+  // split across fewer CTAs, which keeps the number of partials per tile low.
+  long long grid = pl.total_cost / std::max<long long>(kCostSparse, min_cta_weight());
   grid = std::max<long long>(1, std::min<long long>(grid, sms));
   pl.grid = static_cast<int>(grid);
   pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.nsb > 0 ? 256u : 128u);

@@ -102,10 +102,10 @@ def _dev_ptr(t: torch.Tensor | None, dtype, name: str):
 
 
 class _DevView:
-    """Zero-copy view of library-owned device memory for torch.as_tensor."""
+    """Zero-copy view of library-owned device memory for torch.as_tensor (do not write through it)."""
 
     def __init__(self, ptr: int, shape, typestr: str):
-        self.__cuda_array_interface__ = {"data": (ptr, True), "shape": tuple(shape), "typestr": typestr,
+        self.__cuda_array_interface__ = {"data": (ptr, False), "shape": tuple(shape), "typestr": typestr,
                                          "version": 3, "strides": None}
 
 
