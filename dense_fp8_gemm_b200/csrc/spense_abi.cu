@@ -237,6 +237,28 @@ spense_status run_gemm(const spense_packed* Wp, const uint8_t* X, const float* x
   return SPENSE_OK;
 }
 
+// ---------------------------------------------------------------- allocation-free entry point
+// Scratch for spense_gemm_noalloc: a fixed array in device memory that every
+// GPU loading this library holds until the process exits. In host code the
+// symbol is only a stand-in; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SPENSE_NOALLOC_SCRATCH_BYTES];
+
+spense_status noalloc_scratch(int dev, uint8_t** out) {
+  static std::mutex mu;
+  static std::vector<uint8_t*> addr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<int>(addr.size()) <= dev) addr.resize(dev + 1, nullptr);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return SPENSE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -451,6 +473,37 @@ spense_status spense_workspace_status(void* workspace, void* stream_v, uint32_t*
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   *status_out = word;
   return ok();
+}
+
+spense_status spense_gemm_noalloc(const spense_packed* Wp, const uint8_t* X, const float* x_scale,
+                                  int64_t M, uint16_t* Y, void* stream_v) {
+  if (X == nullptr || x_scale == nullptr || Y == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
+  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(x_scale, 4))
+    return fail(SPENSE_ERR_ALIGN, "X and Y must be 16-byte aligned, x_scale 4-byte aligned");
+  if (Wp == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
+  if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  if (dev != Wp->device)
+    return fail(SPENSE_ERR_ARG, "handle was packed on device %d, current device is %d", Wp->device, dev);
+  const GemmPlan pl = make_plan(Wp, M, info.sms);
+  if (pl.ws.total_device > SPENSE_NOALLOC_SCRATCH_BYTES)
+    return fail(SPENSE_ERR_WORKSPACE,
+                "this GEMM needs %zu bytes of scratch; the built-in scratch holds %zu (use spense_gemm "
+                "with a caller workspace, or fewer tokens)",
+                pl.ws.total_device, static_cast<size_t>(SPENSE_NOALLOC_SCRATCH_BYTES));
+  uint8_t* ws = nullptr;
+  st = noalloc_scratch(dev, &ws);
+  if (st != SPENSE_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  // The status word and the arrival counters must start at zero; the array
+  // keeps whatever the previous call left in it.
+  const cudaError_t e = cudaMemsetAsync(ws, 0, pl.ws.partials_off, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
+  st = run_gemm(Wp, X, x_scale, M, Y, ws, pl, stream);
+  return st == SPENSE_OK ? ok() : st;
 }
 
 }  // extern "C"

@@ -27,8 +27,9 @@ PACK_KEEP_CANONICAL = 1
 SYMBOLS = (
     "spense_pack", "spense_gemm", "spense_gemm_workspace_size", "spense_gemm_host",
     "spense_gemm_host_workspace_size", "spense_free", "spense_get_info",
-    "spense_workspace_status", "spense_last_error", "spense_version",
+    "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class SpenseError(RuntimeError):
@@ -69,10 +70,11 @@ def lib() -> ctypes.CDLL:
     L.spense_free.argtypes = [P]
     L.spense_get_info.argtypes = [P, ctypes.POINTER(PackedInfo)]
     L.spense_workspace_status.argtypes = [P, P, ctypes.POINTER(U32)]
+    L.spense_gemm_noalloc.argtypes = [P, P, P, I64, P, P]
     L.spense_last_error.restype = ctypes.c_char_p
     L.spense_version.restype = ctypes.c_char_p
     for name in ("spense_pack", "spense_gemm", "spense_gemm_host", "spense_free", "spense_get_info",
-                 "spense_workspace_status"):
+                 "spense_workspace_status", "spense_gemm_noalloc"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -242,6 +244,19 @@ def gemm_host(pw: PackedWeight, X_host: torch.Tensor, x_scale_host: torch.Tensor
                                   _stream(stream))
     _check(code, "spense_gemm_host")
     return Y_host
+
+
+def gemm_noalloc(pw: PackedWeight, X: torch.Tensor, x_scale: torch.Tensor, Y: torch.Tensor,
+                 stream=None) -> torch.Tensor:
+    """spense_gemm_noalloc: the GEMM without a caller workspace, for callers that
+    cannot allocate device memory when they run it. The library's built-in
+    scratch array stands in for the workspace, so calls must not overlap on the
+    GPU. Y must be preallocated (this call allocates nothing)."""
+    code = lib().spense_gemm_noalloc(pw.handle, _dev_ptr(X, torch.uint8, "X"),
+                                     _dev_ptr(x_scale, torch.float32, "x_scale"), X.shape[0],
+                                     _dev_ptr(Y, torch.bfloat16, "Y"), _stream(stream))
+    _check(code, "spense_gemm_noalloc")
+    return Y
 
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:

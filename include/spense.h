@@ -153,6 +153,35 @@ SPENSE_API spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t
 
 SPENSE_API size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M);
 
+/*
+ * spense_gemm_noalloc — the same GEMM as spense_gemm, for callers that must not
+ * allocate device memory on the call path and so cannot provide a workspace:
+ * for example a plugin inside an inference engine that owns every device
+ * allocation and hands plugins no allocator, or a serving loop that forbids
+ * cudaMalloc after start-up because it can synchronize the device and can fail
+ * under memory pressure in the middle of a request. The paper has no
+ * counterpart to this entry point; it is a deployment convenience.
+ *
+ * Instead of a caller workspace it uses one fixed scratch array of
+ * SPENSE_NOALLOC_SCRATCH_BYTES that the library places in device memory; every
+ * GPU that loads the library holds it until the process exits. Calls whose
+ * workspace need (spense_gemm_workspace_size) exceeds it are rejected with
+ * SPENSE_ERR_WORKSPACE; decode-sized calls (up to a few dozen tokens on the
+ * 32B/36B-class shapes) fit. The call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current), so make that first call before any stream capture. Every
+ * call clears the array's status word and counters on `stream` before the
+ * GEMM. All calls share the one array: calls whose execution can overlap on the
+ * GPU (different streams without ordering between them) race on it and give
+ * wrong results; serialize them. Arguments, layouts and the remaining errors
+ * are those of spense_gemm. Asynchronous on `stream`.
+ */
+#define SPENSE_NOALLOC_SCRATCH_BYTES (8u << 20)
+SPENSE_API spense_status spense_gemm_noalloc(const spense_packed* Wp, const uint8_t* X, const float* x_scale,
+                                             int64_t M, uint16_t* Y, void* stream);
+
 /* Releases the handle and its device buffers (stream-ordered on the stream the
  * handle was packed on). NULL is accepted. */
 SPENSE_API spense_status spense_free(spense_packed* Wp);
