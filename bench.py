@@ -48,12 +48,16 @@ def parse():
 
 
 SHAPES = (("q_proj", 8192, 5120), ("k_proj", 1024, 5120), ("v_proj", 1024, 5120), ("o_proj", 5120, 8192))
+# One step = one layer's attention projections: q, k and v read the same hidden
+# state and run as one grouped launch; o_proj reads the attention output.
+GROUPS = ((0, 1, 2), (3,))
 
 
 def workload_config(args):
     return {
         "workload": f"attn32b q/k/v/o projections, decode M={args.tokens}",
         "shapes": [f"{n}x{k}" for _, n, k in SHAPES],
+        "launches_per_step": "q+k+v grouped (shared input), o_proj",
         "tokens": args.tokens,
         "dense_frac": args.dense_frac,
         "dense_columns": "tail (SpenseGPT)",
@@ -62,14 +66,30 @@ def workload_config(args):
     }
 
 
-def step_bytes(args, Kd_of):
+def step_bytes(args, dense=False):
     from dense_fp8_gemm_b200 import workloads
-    return sum(workloads.algorithmic_bytes(n, k, Kd_of(k), args.tokens) for _, n, k in SHAPES)
+    total = 0
+    for grp in GROUPS:
+        mem = [(SHAPES[i][1], SHAPES[i][2],
+                SHAPES[i][2] if dense else workloads.dense_count(SHAPES[i][2], args.dense_frac)) for i in grp]
+        total += workloads.group_algorithmic_bytes(mem, args.tokens)
+    return total
 
 
-def kd_of(args):
-    from dense_fp8_gemm_b200 import workloads
-    return lambda k: workloads.dense_count(k, args.dense_frac)
+def read_traffic():
+    """DRAM bytes per launch of spense_gemm_kernel from the committed ncu summary,
+    or None when the kernel source has changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "spense_gemm_attn32b_m16_traffic.txt")
+    src = os.path.join(ROOT, "dense_fp8_gemm_b200", "csrc", "gemm_sm100.cu")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        return rec["dram_bytes_per_launch_avg"] if rec["kernel_source_sha256"] == sha else None
+    except Exception:
+        return None
 
 
 def read_peaks():
@@ -153,29 +173,46 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 
-def oracle_sample_rate(args, rows_per_shape: int, budget_s: float, nthreads: int):
-    """Times the CPU oracle (as it stands) on `rows_per_shape` rows of each
-    projection, repeating until `budget_s` elapses. Returns (GB/s, seconds, reps)."""
+def oracle_items(args, rows_per_shape: int):
+    """The bounded sample the CPU oracle runs: `rows_per_shape` output rows of
+    each projection, with the step's activations (q/k/v share one input)."""
     import oracle
     from dense_fp8_gemm_b200 import workloads
     wl = workloads.ATTN32B
-    items = []
-    for i, (_, n, k) in enumerate(SHAPES):
-        w = workloads.make_weight(wl, i, args.dense_frac)
-        rows = np.linspace(0, n - 1, rows_per_shape).astype(np.int64)
-        keep = oracle.pack(w.W[rows], Kd=w.Kd)["keep"]
-        X, s_x = workloads.make_activations(wl, i, args.tokens)
-        items.append((X, s_x, w.W[rows].copy(), w.s_w[rows].copy(), keep, k, w.Kd))
-    byts = sum(workloads.algorithmic_bytes(rows_per_shape, k, kd, args.tokens) for *_, k, kd in items)
+    acts = {0: workloads.make_activations(wl, 0, args.tokens), 3: workloads.make_activations(wl, 3, args.tokens)}
+    items, members = [], []
+    for grp in GROUPS:
+        X, s_x = acts[grp[0]]
+        mem = []
+        for i in grp:
+            w = workloads.make_weight(wl, i, args.dense_frac)
+            rows = np.linspace(0, w.N - 1, rows_per_shape).astype(np.int64)
+            keep = oracle.pack(w.W[rows], Kd=w.Kd)["keep"]
+            items.append((X, s_x, w.W[rows].copy(), w.s_w[rows].copy(), keep))
+            mem.append((rows_per_shape, w.K, w.Kd))
+        members.append(mem)
+    byts = sum(workloads.group_algorithmic_bytes(m, args.tokens) for m in members)
+    return items, byts
+
+
+def oracle_pass(items, nthreads):
+    import oracle
+    for X, s_x, W, s_w, keep in items:
+        oracle.gemm(X, s_x, W, s_w, keep=keep, nthreads=nthreads)
+
+
+def oracle_sample_rate(args, rows_per_shape: int, budget_s: float, nthreads: int):
+    """Times the CPU oracle (as it stands) on the bounded sample, repeating until
+    `budget_s` elapses. Returns (GB/s, seconds, passes)."""
+    items, byts = oracle_items(args, rows_per_shape)
     reps, t0 = 0, time.perf_counter()
     while True:
-        for X, s_x, W, s_w, keep, _, _ in items:
-            oracle.gemm(X, s_x, W, s_w, keep=keep, nthreads=nthreads)
+        oracle_pass(items, nthreads)
         reps += 1
         el = time.perf_counter() - t0
         if el >= budget_s:
             break
-    return byts * reps / el / 1e9, el, reps, byts
+    return byts * reps / el / 1e9, el, reps
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -187,29 +224,15 @@ def run_reference(args):
         return 0
     cores = os.cpu_count() or 1
     rows = 32  # bounded sample per step: 32 output rows of each projection
-    done_bytes = 0
-    import oracle as _o
-    from dense_fp8_gemm_b200 import workloads as _w
-    wl = _w.ATTN32B
-    items = []
-    for i, (_, n, k) in enumerate(SHAPES):
-        w = _w.make_weight(wl, i, args.dense_frac)
-        r = np.linspace(0, n - 1, rows).astype(np.int64)
-        keep = _o.pack(w.W[r], Kd=w.Kd)["keep"]
-        X, s_x = _w.make_activations(wl, i, args.tokens)
-        items.append((X, s_x, w.W[r].copy(), w.s_w[r].copy(), keep, k, w.Kd))
-    per_step = sum(_w.algorithmic_bytes(rows, k, kd, args.tokens) for *_, k, kd in items)
+    items, per_step = oracle_items(args, rows)
     for _ in range(args.warmup):
-        for X, s_x, W, s_w, keep, _, _ in items:
-            _o.gemm(X, s_x, W, s_w, keep=keep, nthreads=cores)
+        oracle_pass(items, cores)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        for X, s_x, W, s_w, keep, _, _ in items:
-            _o.gemm(X, s_x, W, s_w, keep=keep, nthreads=cores)
-        done_bytes += per_step
+        oracle_pass(items, cores)
     el = time.perf_counter() - t0
-    value = done_bytes / el / 1e9
-    sample = f"{rows} rows of each of q/k/v/o per step (M={args.tokens}); full rows scale linearly"
+    value = per_step * args.steps / el / 1e9
+    sample = f"{rows} output rows of each of q/k/v/o per step (M={args.tokens}), all {cores} host threads"
     line = {
         "impl": "reference", "metric": "spense_fp8_weight_stream_GBps", "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -238,18 +261,12 @@ def run_spense(args):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    stream = torch.cuda.current_stream()
 
     M = args.tokens
-    Kd_of = kd_of(args)
     wl = workloads.ATTN32B
     # ---- weights: one synthetic layer, packed into `layers` distinct buffer sets
-    layers_sp, layers_dn, dims = [], [], []
-    host_w = []
-    for i, (_, n, k) in enumerate(SHAPES):
-        w = workloads.make_weight(wl, i, args.dense_frac)
-        host_w.append(w)
-        dims.append((n, k, w.Kd))
+    host_w = [workloads.make_weight(wl, i, args.dense_frac) for i in range(len(SHAPES))]
+    layers_sp, layers_dn = [], []
     for _ in range(args.layers):
         sp, dn = [], []
         for w in host_w:
@@ -260,35 +277,35 @@ def run_spense(args):
             del Wd
         layers_sp.append(sp)
         layers_dn.append(dn)
-    acts = []
-    for i in range(len(SHAPES)):
-        X, s_x = workloads.make_activations(wl, i, M)
-        acts.append((torch.from_numpy(X).to(dev), torch.from_numpy(s_x).to(dev), X, s_x))
-    Ys = [torch.empty((M, n), dtype=torch.bfloat16, device=dev) for n, _, _ in dims]
-    ws_bytes = max(spense.workspace_size(p, M) for L in (layers_sp, layers_dn) for p in L[0])
+    # activations: q/k/v share the hidden state, o_proj reads the attention output
+    host_x = {grp[0]: workloads.make_activations(wl, grp[0], M) for grp in GROUPS}
+    dev_x = {k: (torch.from_numpy(v[0]).to(dev), torch.from_numpy(v[1]).to(dev)) for k, v in host_x.items()}
+    Ys = [torch.empty((M, n), dtype=torch.bfloat16, device=dev) for _, n, _ in SHAPES]
+    ws_bytes = max(spense.grouped_workspace_size([L[i] for i in grp], M)
+                   for L in (layers_sp[0], layers_dn[0]) for grp in GROUPS)
     ws = spense.new_workspace(ws_bytes, dev)
     torch.cuda.synchronize()
 
-    def launch_layer(layer_packs):
-        for s, pw in enumerate(layer_packs):
-            spense.gemm(pw, acts[s][0], acts[s][1], Ys[s], ws, stream)
+    def launch_layer(packs, stream, events=None):
+        for gi, grp in enumerate(GROUPS):
+            X, sx = dev_x[grp[0]]
+            if events is not None:
+                events[gi][0].record(stream)
+            spense.gemm_grouped([packs[i] for i in grp], X, sx, [Ys[i] for i in grp], ws, stream)
+            if events is not None:
+                events[gi][1].record(stream)
 
     def capture(layer_list, with_events=False):
         graphs, evs = [], []
         for L in layer_list:
-            launch_layer(L)  # warm (attribute setup outside capture)
+            launch_layer(L, torch.cuda.current_stream())  # warm (attribute setup outside capture)
         torch.cuda.synchronize()
         for L in layer_list:
             g = torch.cuda.CUDAGraph()
             e = [(torch.cuda.Event(enable_timing=True, external=True),
-                  torch.cuda.Event(enable_timing=True, external=True)) for _ in L] if with_events else None
+                  torch.cuda.Event(enable_timing=True, external=True)) for _ in GROUPS] if with_events else None
             with torch.cuda.graph(g):
-                for s, pw in enumerate(L):
-                    if with_events:
-                        e[s][0].record()
-                    spense.gemm(pw, acts[s][0], acts[s][1], Ys[s], ws, torch.cuda.current_stream())
-                    if with_events:
-                        e[s][1].record()
+                launch_layer(L, torch.cuda.current_stream(), e)
             graphs.append(g)
             evs.append(e)
         torch.cuda.synchronize()
@@ -327,43 +344,54 @@ def run_spense(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         t_sp, t_dn = t.tolist()
 
-    per_step = step_bytes(args, Kd_of)
+    per_step = step_bytes(args)
     value = per_step * args.steps * world / t_sp / 1e9
-    launches = args.steps * len(SHAPES)
+    launches = args.steps * len(GROUPS)
 
-    # ---- dominant kernel: per-launch device time from events captured around each GEMM
+    # ---- dominant kernel: per-launch device time from events captured around each launch
     g_ev, evs = capture(layers_sp, with_events=True)
-    dur = [[] for _ in SHAPES]
+    dur = [[] for _ in GROUPS]
     reps = max(8, min(args.steps, 64))
     for i in range(reps):
         g_ev[i % len(g_ev)].replay()
         torch.cuda.synchronize()
-        for s, (a, b) in enumerate(evs[i % len(g_ev)]):
-            dur[s].append(a.elapsed_time(b) / 1e3)
-    per_launch = [statistics.median(d) for d in dur]
-    bytes_per_launch = [workloads.algorithmic_bytes(n, k, kd, M) for n, k, kd in dims]
-    achieved = sum(bytes_per_launch) / sum(per_launch) / 1e9
+        for gi, (a, b) in enumerate(evs[i % len(g_ev)]):
+            dur[gi].append(a.elapsed_time(b) / 1e3)
+    per_launch = [statistics.median(d) for d in dur]  # isolated: event nodes serialize the launches
+    # The timed region holds only spense_gemm_kernel launches (tail dense set: no gather), so the
+    # average launch duration over it is t_sp / launches and the bytes per launch average the
+    # step's algorithmic bytes over its launches.
+    avg_launch_s = t_sp / launches
+    bytes_per_launch = per_step / len(GROUPS)
+    achieved = bytes_per_launch / avg_launch_s / 1e9
     peak, peak_kind = read_peaks()
     del g_ev, evs
 
-    # ---- e2e through the host-buffer entry point (copies inside the timed region)
-    hws = spense.new_workspace(max(spense.host_workspace_size(p, M) for p in layers_sp[0]), dev)
-    hx = [torch.from_numpy(a[2]).pin_memory() for a in acts]
-    hs = [torch.from_numpy(a[3]).pin_memory() for a in acts]
-    hy = [torch.empty((M, n), dtype=torch.bfloat16).pin_memory() for n, _, _ in dims]
-    e2e_steps = max(4, min(args.steps, 100))
-    for i in range(min(args.warmup, 4)):
-        for s, pw in enumerate(layers_sp[i % args.layers]):
-            spense.gemm_host(pw, hx[s], hs[s], hy[s], hws, stream)
-    torch.cuda.synchronize()
+    # ---- e2e: host buffers in, host buffers out, copies inside the timed region
+    hx = {k: (torch.from_numpy(v[0]).pin_memory(), torch.from_numpy(v[1]).pin_memory()) for k, v in host_x.items()}
+    hy = [torch.empty((M, n), dtype=torch.bfloat16).pin_memory() for _, n, _ in SHAPES]
+    stream = torch.cuda.current_stream()
+
+    def e2e_step(packs):
+        for grp in GROUPS:
+            X, sx = dev_x[grp[0]]
+            X.copy_(hx[grp[0]][0], non_blocking=True)
+            sx.copy_(hx[grp[0]][1], non_blocking=True)
+            spense.gemm_grouped([packs[i] for i in grp], X, sx, [Ys[i] for i in grp], ws, stream)
+            for i in grp:
+                hy[i].copy_(Ys[i], non_blocking=True)
+        stream.synchronize()
+
+    e2e_steps = max(4, min(args.steps, 200))
+    for i in range(min(args.warmup, 8)):
+        e2e_step(layers_sp[i % args.layers])
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(e2e_steps):
-        for s, pw in enumerate(layers_sp[i % args.layers]):
-            spense.gemm_host(pw, hx[s], hs[s], hy[s], hws, stream)
+        e2e_step(layers_sp[i % args.layers])
     e1.record()
     torch.cuda.synchronize()
     t_e2e = e0.elapsed_time(e1) / 1e3
@@ -371,8 +399,8 @@ def run_spense(args):
         t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         t_e2e = t.item()
-    h2d = sum(M * k + 4 * M for _, k, _ in dims)
-    d2h = sum(2 * M * n for n, _, _ in dims)
+    h2d = sum(M * SHAPES[g[0]][2] + 4 * M for g in GROUPS)
+    d2h = sum(2 * M * n for _, n, _ in SHAPES)
     e2e_value = per_step * e2e_steps * world / t_e2e / 1e9
 
     status = spense.workspace_status(ws)
@@ -382,25 +410,27 @@ def run_spense(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cores = os.cpu_count() or 1
-        gbs, el, reps_c, byts = oracle_sample_rate(args, 256, args.cpu_seconds, cores)
+        gbs, el, reps_c = oracle_sample_rate(args, 256, args.cpu_seconds, cores)
         cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": f"256 rows of each of q/k/v/o, M={args.tokens}, {reps_c} passes in {el:.1f} s"}
+               "sample": f"256 output rows of each of q/k/v/o, M={args.tokens}, {reps_c} passes in {el:.1f} s"}
 
     if rank == 0:
-        tflops = sum(workloads.useful_flops(n, k, kd, M) for n, k, kd in dims) * args.steps * world / t_sp / 1e12
+        kd = [workloads.dense_count(k, args.dense_frac) for _, _, k in SHAPES]
+        tflops = sum(workloads.useful_flops(n, k, kd[i], M) for i, (_, n, k) in enumerate(SHAPES)) \
+            * args.steps * world / t_sp / 1e12
         line = {
             "metric": "spense_fp8_weight_stream_GBps", "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_sp / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe4m3->f32",
             "data": "synthetic", "config": workload_config(args),
             "speedup_vs_dense_fp8": t_dn / t_sp,
-            "dense_fp8_GBps": (sum(workloads.algorithmic_bytes(n, k, k, M) for n, k, _ in dims)
-                               * args.steps * world / t_dn / 1e9),
+            "dense_fp8_GBps": step_bytes(args, dense=True) * args.steps * world / t_dn / 1e9,
             "tflops": tflops,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_source": peak_kind,
-                         "kernel": "spense_gemm_kernel",
-                         "per_launch_us": {SHAPES[s][0]: per_launch[s] * 1e6 for s in range(len(SHAPES))}},
+                         "frac": achieved / peak, "traffic": read_traffic(), "peak_source": peak_kind,
+                         "kernel": "spense_gemm_kernel", "avg_launch_us": avg_launch_s * 1e6,
+                         "bytes_per_launch": bytes_per_launch,
+                         "isolated_launch_us": {"qkv_grouped": per_launch[0] * 1e6, "o_proj": per_launch[1] * 1e6}},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,

@@ -10,7 +10,10 @@
 //
 // Layout of the work (swap-AB): weight rows are the MMA M dimension (128 per
 // tile), tokens are the MMA N dimension (padded to a multiple of 16), K is the
-// packed column order (2:4 region first, then the dense region).
+// packed column order (2:4 region first, then the dense region). Up to
+// kMaxGroup weight matrices with the same K layout can share one launch and
+// one activation tensor (for example q, k and v projections); their row tiles
+// are laid end to end.
 //
 // Roles (one CTA per SM, 192 threads):
 //   warp 0   producer: bulk copies of the packed weight blocks (values,
@@ -23,9 +26,11 @@
 //
 // Work split ("stream-K by bytes"): the blocks of all tiles form one sequence,
 // each block weighted by the HBM bytes it streams (a 2:4 block 20 KiB, a dense
-// block 16 KiB). CTA g takes the blocks whose start falls in
-// [g T / G, (g+1) T / G) of the total weight T. A tile split across CTAs is
-// finished by the last CTA to arrive, which sums every contributor's partial in
+// block 16 KiB). The host cuts the sequence into one contiguous range per CTA
+// (p.cta_start). A CTA handles the tiles it shares with its neighbours first
+// and its whole tiles last, so the cross-CTA fix-ups overlap the streaming of
+// whole tiles instead of forming the kernel's tail. A shared tile is finished
+// by the last contributor to arrive, which sums every contributor's partial in
 // CTA order, so the result does not depend on arrival order.
 //
 // Every wait is bounded (1.5 s by %globaltimer); on expiry the kernel records a
@@ -71,77 +76,78 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, unsigned
   }
 }
 
-// ---------------------------------------------------------------- work split
-struct Split {
-  const GemmParams& p;
-  int nblk;
-  __device__ explicit Split(const GemmParams& pp) : p(pp), nblk(pp.nsb + pp.ndb) {}
-
-  // Start weight of block j inside a tile.
-  __device__ long long block_start(int j) const {
-    return j <= p.nsb ? static_cast<long long>(kCostSparse) * j
-                      : static_cast<long long>(kCostSparse) * p.nsb +
-                            static_cast<long long>(kCostDense) * (j - p.nsb);
-  }
-  // First linear block (tile * nblk + j) whose start weight is >= c.
-  __device__ long long first_block_at(long long c) const {
-    const long long t = c / p.tile_cost;
-    const long long r = c - t * p.tile_cost;
-    const long long sp = static_cast<long long>(kCostSparse) * p.nsb;
-    long long j;
-    if (r <= sp)
-      j = (r + kCostSparse - 1) / kCostSparse;
+// CTA owning linear block b: the last g with cta_start[g] <= b.
+__device__ __forceinline__ int block_owner(const GemmParams& p, int b) {
+  int lo = 0, hi = p.grid - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.cta_start[mid] <= b)
+      lo = mid;
     else
-      j = p.nsb + (r - sp + kCostDense - 1) / kCostDense;
-    return t * nblk + j;
+      hi = mid - 1;
   }
-  __device__ long long cta_start_weight(int g) const {
-    return (static_cast<long long>(g) * p.total_cost + p.grid - 1) / p.grid;
+  return lo;
+}
+
+// The units (tile, block range) of one CTA's block range, in processing order:
+// a partial last unit is moved to the front, so both shared tiles come first.
+struct Units {
+  int nblk, t_first, j_first, t_last, j_last_end, count;
+  bool move_last;
+  __device__ Units(int b0, int b1, int nblk_) : nblk(nblk_) {
+    if (b1 <= b0) {
+      count = 0;
+      t_first = j_first = t_last = j_last_end = 0;
+      move_last = false;
+      return;
+    }
+    t_first = b0 / nblk;
+    j_first = b0 - t_first * nblk;
+    t_last = (b1 - 1) / nblk;
+    j_last_end = b1 - t_last * nblk;
+    count = t_last - t_first + 1;
+    move_last = count >= 2 && j_last_end < nblk;
   }
-  __device__ long long cta_first_block(int g) const { return first_block_at(cta_start_weight(g)); }
-  // CTA owning block j of tile t.
-  __device__ int owner(long long t, int j) const {
-    const long long s = t * p.tile_cost + block_start(j);
-    return static_cast<int>((s * p.grid) / p.total_cost);
+  // Unit at processing position u: tile t, blocks [j0, j1).
+  __device__ void get(int u, int& t, int& j0, int& j1) const {
+    const int k = move_last ? (u == 0 ? count - 1 : u - 1) : u;
+    t = t_first + k;
+    j0 = (k == 0) ? j_first : 0;
+    j1 = (k == count - 1) ? j_last_end : nblk;
   }
-  // Partial slot CTA g uses for tile t: 0 for its first tile, 1 for its last.
-  __device__ int slot(int g, long long t) const { return (cta_first_block(g) / nblk == t) ? 0 : 1; }
 };
 
-// Iterates the units (t, j0, j1) of a block range.
-struct UnitIter {
-  long long b, b1;
-  int nblk;
-  __device__ UnitIter(long long b0_, long long b1_, int nblk_) : b(b0_), b1(b1_), nblk(nblk_) {}
-  __device__ bool next(long long& t, int& j0, int& j1) {
-    if (b >= b1) return false;
-    t = b / nblk;
-    j0 = static_cast<int>(b - t * nblk);
-    const long long left = b1 - b;
-    j1 = static_cast<int>(left < nblk - j0 ? j0 + left : nblk);
-    b += j1 - j0;
-    return true;
-  }
-};
+// Group member holding global row tile n_tile.
+__device__ __forceinline__ int member_of(const GemmParams& p, int n_tile) {
+  int i = 0;
+#pragma unroll
+  for (int k = 1; k < kMaxGroup; ++k)
+    if (k < p.n_members && p.mem[k].tile_begin <= n_tile) i = k;
+  return i;
+}
 
-// Walks blocks b0, b0+1, ... keeping (tile, block, n-tile, token-tile)
-// incrementally, so the per-block path has no integer division.
-struct BlockCursor {
-  int j, nblk, m_tile, m_tiles;
-  long long n_tile;
-  __device__ BlockCursor(long long b, int nblk_, int m_tiles_) : nblk(nblk_), m_tiles(m_tiles_) {
-    const long long t = b / nblk;
-    j = static_cast<int>(b - t * nblk);
-    n_tile = t / m_tiles;
-    m_tile = static_cast<int>(t - n_tile * m_tiles);
+// Walks the blocks of a CTA in processing order without integer division on
+// the per-block path.
+struct BlockWalker {
+  const Units* units;
+  int u, j, j1, m_tile, m_tiles, member, local_tile;
+  __device__ BlockWalker(const Units& us, const GemmParams& p) : units(&us), u(0), m_tiles(p.m_tiles) {
+    enter(p);
   }
-  __device__ void advance() {
-    if (++j == nblk) {
-      j = 0;
-      if (++m_tile == m_tiles) {
-        m_tile = 0;
-        ++n_tile;
-      }
+  __device__ void enter(const GemmParams& p) {
+    if (u >= units->count) return;
+    int t, j0;
+    units->get(u, t, j0, j1);
+    j = j0;
+    const int n_tile = t / m_tiles;
+    m_tile = t - n_tile * m_tiles;
+    member = member_of(p, n_tile);
+    local_tile = n_tile - p.mem[member].tile_begin;
+  }
+  __device__ void advance(const GemmParams& p) {
+    if (++j == j1) {
+      ++u;
+      enter(p);
     }
   }
 };
@@ -162,8 +168,8 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
-__global__ void __launch_bounds__(kGemmThreads, 1)
-    spense_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const GemmParams p) {
+__global__ void __launch_bounds__(kGemmThreadsMax, 2)
+    spense_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -201,38 +207,48 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // anything this grid writes.
   ptx::griddep_launch_dependents();
 
-  const Split split(p);
-  const long long b0 = split.cta_first_block(g);
-  const long long b1 = split.cta_first_block(g + 1);
+  const int nblk = p.nsb + p.ndb;
+  const int b0 = p.cta_start[g];
+  const int b1 = p.cta_start[g + 1];
+  const Units units(b0, b1, nblk);
   const uint32_t smem_base = ptx::smem_addr(smem);
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    // Blocks b0..b1-1 go through the ring in order. The weight copies of the
-    // first ring's worth are issued before waiting on the previous grid (the
-    // packed weights never depend on it), the activation tiles after.
+  if (warp == 0 || warp == 6) {
+    // ------------------------------------------------------------ producer(s)
+    // Blocks go through the ring in processing order. The weight copies of
+    // the first ring's worth are issued before waiting on the previous grid
+    // (the packed weights never depend on it), the activation tiles after.
+    // With two producer warps (warps 0 and 6) each issues every other block:
+    // the copy engine serves the two issue streams concurrently.
     if (lane == 0) {
+      const int np = p.producers;
+      const int me = warp == 0 ? 0 : 1;
       const uint64_t pol_w = ptx::policy_evict_first();
       const uint64_t pol_x = ptx::policy_evict_last();
-      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
-      const long long nb = b1 - b0;
-      const int pre = static_cast<int>(nb < p.stages ? nb : p.stages);
-      auto issue_w = [&](const BlockCursor& c, uint32_t s) {
+      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;         // smem bytes of a K-atom
+      const uint32_t xbytes = static_cast<uint32_t>(p.box_rows) * 128u;  // bytes one TMA box loads
+      const int nb = b1 - b0;
+      const int pre = nb < p.stages ? nb : p.stages;
+      auto issue_w = [&](const BlockWalker& c, uint32_t s) {
+        const GemmMember& mb = p.mem[c.member];
         const uint32_t a_s = smem_base + s * p.stage_bytes;
         const uint32_t full = ptx::smem_addr(&bars->full[s]);
+        const uint32_t piece = kBlockBytes / static_cast<uint32_t>(p.bulk_split);
         if (c.j < p.nsb) {
-          const size_t blk = static_cast<size_t>(c.n_tile) * p.nsb + c.j;
-          ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * box);
-          ptx::bulk_g2s(a_s, p.vs_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
-          ptx::bulk_g2s(a_s + kBlockBytes + p.b_bytes, p.e_t + blk * kMetaBlockBytes, kMetaBlockBytes, full,
-                        pol_w);
+          const size_t blk = static_cast<size_t>(c.local_tile) * p.nsb + c.j;
+          ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * xbytes);
+          for (int q = 0; q < p.bulk_split; ++q)
+            ptx::bulk_g2s(a_s + q * piece, mb.vs_t + blk * kBlockBytes + q * piece, piece, full, pol_w);
+          ptx::bulk_g2s(a_s + kBlockBytes + p.b_bytes, mb.e_t + blk * kMetaBlockBytes, kMetaBlockBytes,
+                        full, pol_w);
         } else {
-          const size_t blk = static_cast<size_t>(c.n_tile) * p.ndb + (c.j - p.nsb);
-          ptx::mbar_arrive_expect_tx(full, kBlockBytes + box);
-          ptx::bulk_g2s(a_s, p.wd_t + blk * kBlockBytes, kBlockBytes, full, pol_w);
+          const size_t blk = static_cast<size_t>(c.local_tile) * p.ndb + (c.j - p.nsb);
+          ptx::mbar_arrive_expect_tx(full, kBlockBytes + xbytes);
+          for (int q = 0; q < p.bulk_split; ++q)
+            ptx::bulk_g2s(a_s + q * piece, mb.wd_t + blk * kBlockBytes + q * piece, piece, full, pol_w);
         }
       };
-      auto issue_x = [&](const BlockCursor& c, uint32_t s) {
+      auto issue_x = [&](const BlockWalker& c, uint32_t s) {
         const int y0 = c.m_tile * kMaxTokenTile;
         const uint32_t b_s = smem_base + s * p.stage_bytes + kBlockBytes;
         const uint32_t full = ptx::smem_addr(&bars->full[s]);
@@ -243,14 +259,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           ptx::tma_load_2d(b_s, &tmap_x, p.Ks + (c.j - p.nsb) * kDenseBlockCols, y0, full, pol_x);
         }
       };
-      BlockCursor cw(b0, split.nblk, p.m_tiles);
-      for (int i = 0; i < pre; ++i, cw.advance()) issue_w(cw, static_cast<uint32_t>(i));
+      BlockWalker cw(units, p);
+      for (int i = 0; i < pre; ++i, cw.advance(p))
+        if (i % np == me) issue_w(cw, static_cast<uint32_t>(i));
       ptx::griddep_wait();
-      BlockCursor cx(b0, split.nblk, p.m_tiles);
-      for (int i = 0; i < pre; ++i, cx.advance()) issue_x(cx, static_cast<uint32_t>(i));
+      BlockWalker cx(units, p);
+      for (int i = 0; i < pre; ++i, cx.advance(p))
+        if (i % np == me) issue_x(cx, static_cast<uint32_t>(i));
       Ring ring(static_cast<uint32_t>(p.stages));
       for (int i = 0; i < pre; ++i) ring.advance();
-      for (long long i = pre; i < nb; ++i, ring.advance(), cw.advance()) {
+      for (int i = pre; i < nb; ++i, ring.advance(), cw.advance(p)) {
+        if (i % np != me) continue;
         if (!wait_bar(ptx::smem_addr(&bars->empty[ring.s]), ring.ph ^ 1u, p.status,
                       SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag))
           break;
@@ -264,15 +283,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t idesc_sp = ptx::idesc_f8(static_cast<uint32_t>(p.npad), true);
       const uint32_t idesc_d = ptx::idesc_f8(static_cast<uint32_t>(p.npad), false);
       const uint32_t e_col0 = static_cast<uint32_t>(p.nacc * p.npad);
-      UnitIter units(b0, b1, split.nblk);
-      long long t;
-      int j0, j1;
-      uint32_t u = 0, ebuf = 0;
+      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
       Ring ring(static_cast<uint32_t>(p.stages));
+      uint32_t ebuf = 0;
       bool ok = true;
-      while (ok && units.next(t, j0, j1)) {
-        const uint32_t acc = u % p.nacc;
-        const uint32_t aph = (u / p.nacc) & 1u;
+      for (int u = 0; ok && u < units.count; ++u) {
+        int t, j0, j1;
+        units.get(u, t, j0, j1);
+        const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
+        const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
         if (!wait_bar(ptx::smem_addr(&bars->acc_empty[acc]), aph ^ 1u, p.status,
                       SPENSE_DEVICE_TIMEOUT_MMA, abort_flag)) {
           ok = false;
@@ -281,18 +300,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.npad);
         for (int j = j0; j < j1; ++j, ring.advance()) {
-          const uint32_t s = ring.s;
-          const uint32_t ph = ring.ph;
-          if (!wait_bar(ptx::smem_addr(&bars->full[s]), ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
+          if (!wait_bar(ptx::smem_addr(&bars->full[ring.s]), ring.ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
                         abort_flag)) {
             ok = false;
             break;
           }
           ptx::tc_fence_after();
-          const uint32_t a_s = smem_base + s * p.stage_bytes;
+          const uint32_t a_s = smem_base + ring.s * p.stage_bytes;
           const uint32_t b_s = a_s + kBlockBytes;
           const uint32_t e_s = b_s + p.b_bytes;
-          const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
           if (j < p.nsb) {
             const uint32_t e_tmem = tmem_base + e_col0 + ebuf * 8u;
             ptx::tmem_cp_128x128b(e_tmem, ptx::desc_rows16(e_s));
@@ -301,8 +317,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (uint32_t k = 0; k < 4; ++k) {
               const uint64_t ad = ptx::desc_sw128(a_s + 32u * k);
               const uint64_t bd = ptx::desc_sw128(b_s + (k >> 1) * box + (k & 1u) * 64u);
-              ptx::mma_sp_f8(d_tmem, ad, bd, e_tmem + 2u * k, idesc_sp,
-                             (j > j0 || k > 0) ? 1u : 0u);
+              ptx::mma_sp_f8(d_tmem, ad, bd, e_tmem + 2u * k, idesc_sp, (j > j0 || k > 0) ? 1u : 0u);
             }
             ebuf ^= 1u;
           } else {
@@ -313,43 +328,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               ptx::mma_f8(d_tmem, ad, bd, idesc_d, (j > j0 || k > 0) ? 1u : 0u);
             }
           }
-          ptx::mma_commit(ptx::smem_addr(&bars->empty[s]));
+          ptx::mma_commit(ptx::smem_addr(&bars->empty[ring.s]));
         }
         if (!ok) break;
         ptx::mma_commit(ptx::smem_addr(&bars->acc_full[acc]));
-        ++u;
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
     ptx::griddep_wait();  // s_x, Y and the workspace may belong to the previous grid
-    const int et = threadIdx.x - 64;           // 0..127
-    const int quarter = warp & 3;              // tensor-memory lane quarter this warp may read
+    const int et = threadIdx.x - 64;  // 0..127
+    const int quarter = warp & 3;     // tensor-memory lane quarter this warp may read
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
-    UnitIter units(b0, b1, split.nblk);
-    long long t;
-    int j0, j1;
-    uint32_t u = 0;
-    while (units.next(t, j0, j1)) {
-      const uint32_t acc = u % p.nacc;
-      const uint32_t aph = (u / p.nacc) & 1u;
+    const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
+    for (int u = 0; u < units.count; ++u) {
+      int t, j0, j1;
+      units.get(u, t, j0, j1);
+      const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
+      const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
       const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
       if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
       ptx::tc_fence_after();
-      const long long n_tile = t / p.m_tiles;
-      const int m0 = static_cast<int>(t % p.m_tiles) * kMaxTokenTile;
+      const int n_tile = t / p.m_tiles;
+      const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
-      const int n = static_cast<int>(n_tile) * kTileRows + row;
-      const bool row_ok = n < p.N;
-      const float sw = row_ok ? __ldg(p.s_w + n) : 0.0f;
-      const bool whole = (j0 == 0 && j1 == split.nblk);
+      const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+      const bool row_ok = n < mb.N;
+      const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
+      const bool whole = (j0 == 0 && j1 == nblk);
       const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
-      // Partials are stored [slot][row][npad] so each thread owns one contiguous row.
+      // Partials are stored [CTA][slot][row][npad]: slot 0 for the tile holding the
+      // CTA's first block, slot 1 for the tile holding its last block.
       float* part = nullptr;
-      if (!whole)
-        part = p.partials + ((static_cast<size_t>(g) * 2 + split.slot(g, t)) * kTileRows + row) * p.npad;
+      if (!whole) {
+        const int slot = (b0 >= t * nblk) ? 0 : 1;
+        part = p.partials + (static_cast<size_t>(g) * 2 + slot) * slot_elems + static_cast<size_t>(row) * p.npad;
+      }
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
         uint32_t v[16];
         ptx::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), v);
@@ -360,7 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int i = 0; i < 16; ++i) {
               const int m = c0 + i;
               if (m < m_valid)
-                p.y[static_cast<size_t>(m0 + m) * p.N + n] =
+                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] =
                     to_bf16_bits(__uint_as_float(v[i]) * sw * __ldg(p.s_x + m0 + m));
             }
           }
@@ -375,80 +392,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
-      ++u;
-      if (!whole) {
-        // Publish this CTA's partial: the named barrier orders the 128 threads'
-        // stores before thread 0's release-acquire ticket at GPU scope.
-        ptx::named_bar_sync(1, 128);
-        const int g_lo = split.owner(t, 0);
-        const int g_hi = split.owner(t, split.nblk - 1);
-        if (et == 0) {
-          const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
-          bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
+      if (whole) continue;
+
+      // Publish this CTA's partial: the named barrier orders the 128 threads'
+      // stores before thread 0's release-acquire ticket at GPU scope.
+      ptx::named_bar_sync(1, 128);
+      const int g_lo = block_owner(p, t * nblk);
+      const int g_hi = block_owner(p, t * nblk + nblk - 1);
+      if (et == 0) {
+        const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
+        bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
+      }
+      ptx::named_bar_sync(1, 128);
+      if (!*reinterpret_cast<volatile int*>(&bars->fix_flag)) continue;
+
+      // Last to arrive: sum the contributors' partials in CTA order. Every
+      // contributor after g_lo starts inside tile t, so its partial is in slot
+      // 0; g_lo uses slot 1 when its range started in an earlier tile.
+      const int lo_slot = (p.cta_start[g_lo] >= t * nblk) ? 0 : 1;
+      const float* lo_part =
+          p.partials + (static_cast<size_t>(g_lo) * 2 + lo_slot) * slot_elems + static_cast<size_t>(row) * p.npad;
+      const float* next_part =
+          p.partials + (static_cast<size_t>(g_lo + 1) * 2) * slot_elems + static_cast<size_t>(row) * p.npad;
+      const size_t stride = 2 * slot_elems;  // from contributor gg to gg + 1 (slot 0)
+      const int others = g_hi - g_lo;
+      for (int c0 = 0; c0 < m_valid; c0 += 16) {
+        const int nq = min(4, (m_valid - c0 + 3) >> 2);  // float4 groups holding valid tokens
+        float4 a[4], b[4], c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nq) a[q] = __ldcg(reinterpret_cast<const float4*>(lo_part + c0) + q);
+        int k = 0;
+        for (; k + 2 <= others; k += 2) {
+          const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
+          const float4* pc = reinterpret_cast<const float4*>(next_part + (k + 1) * stride + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < nq) {
+              b[q] = __ldcg(pb + q);
+              c[q] = __ldcg(pc + q);
+            }
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (q < nq) {
+              a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
+              a[q].x += c[q].x; a[q].y += c[q].y; a[q].z += c[q].z; a[q].w += c[q].w;
+            }
         }
-        ptx::named_bar_sync(1, 128);
-        const int finisher = *reinterpret_cast<volatile int*>(&bars->fix_flag);
-        if (finisher) {
-          // Contributors g_lo..g_hi own consecutive block ranges of tile t. Every
-          // contributor after g_lo starts inside t, so its partial is in slot 0;
-          // g_lo uses slot 1 when its range started in an earlier tile. The sum
-          // runs in contributor order.
-          const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
-          const float* lo_part =
-              p.partials + (static_cast<size_t>(g_lo) * 2 + split.slot(g_lo, t)) * slot_elems +
-              static_cast<size_t>(row) * p.npad;
-          const float* next_part =
-              p.partials + (static_cast<size_t>(g_lo + 1) * 2) * slot_elems + static_cast<size_t>(row) * p.npad;
-          const size_t stride = 2 * slot_elems;  // from contributor gg to gg + 1 (slot 0)
-          const int others = g_hi - g_lo;
-          for (int c0 = 0; c0 < m_valid; c0 += 16) {
-            const int nq = min(4, (m_valid - c0 + 3) >> 2);  // float4 groups holding valid tokens
-            float4 a[4], b[4], c[4];
+        if (k < others) {
+          const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              if (q < nq) a[q] = __ldcg(reinterpret_cast<const float4*>(lo_part + c0) + q);
-            int k = 0;
-            for (; k + 2 <= others; k += 2) {
-              const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
-              const float4* pc = reinterpret_cast<const float4*>(next_part + (k + 1) * stride + c0);
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                if (q < nq) {
-                  b[q] = __ldcg(pb + q);
-                  c[q] = __ldcg(pc + q);
-                }
-#pragma unroll
-              for (int q = 0; q < 4; ++q)
-                if (q < nq) {
-                  a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
-                  a[q].x += c[q].x; a[q].y += c[q].y; a[q].z += c[q].z; a[q].w += c[q].w;
-                }
+          for (int q = 0; q < 4; ++q)
+            if (q < nq) {
+              b[q] = __ldcg(pb + q);
+              a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
             }
-            if (k < others) {
-              const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
+        }
+        if (row_ok) {
 #pragma unroll
-              for (int q = 0; q < 4; ++q)
-                if (q < nq) {
-                  b[q] = __ldcg(pb + q);
-                  a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
-                }
-            }
-            if (row_ok) {
+          for (int q = 0; q < 4; ++q) {
+            const float r4[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float r4[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int m = c0 + 4 * q + i;
-                  if (q < nq && m < m_valid)
-                    p.y[static_cast<size_t>(m0 + m) * p.N + n] = to_bf16_bits(r4[i] * sw * __ldg(p.s_x + m0 + m));
-                }
-              }
+            for (int i = 0; i < 4; ++i) {
+              const int m = c0 + 4 * q + i;
+              if (q < nq && m < m_valid)
+                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(r4[i] * sw * __ldg(p.s_x + m0 + m));
             }
           }
-          if (et == 0) atomicExch(p.counters + t, 0u);
         }
       }
+      if (et == 0) p.counters[t] = 0u;  // re-arm for the next launch (ordered by the kernel boundary)
     }
   }
 
@@ -486,7 +499,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
   }();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(p.grid));
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(kGemmThreads + 32 * (p.producers - 1));
   cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -26,6 +26,7 @@ struct spense_packed {
   uint8_t* wd_t = nullptr;
   float* s_w = nullptr;
   int32_t* perm = nullptr;
+  std::vector<int32_t> perm_host;  // same order on the host (empty for the tail)
   uint8_t* vs_c = nullptr;
   uint8_t* e_c = nullptr;
   uint8_t* wd_c = nullptr;
@@ -121,33 +122,103 @@ long long min_cta_weight() {
   return v;
 }
 
-// Launch plan for (handle, M) on a device with `sms` SMs.
-GemmPlan make_plan(const spense_packed* h, int64_t M, int sms) {
+// Tuning knobs read once from the environment: CTAs per SM (1 or 2, default 2),
+// loader warps per CTA (1 or 2, default 2) and how many bulk copies move one
+// 16 KiB weight block (1, 2 or 4, default 1). One SM's copy engine serves
+// several issue streams at once but one stream's copies one after another, so
+// two CTAs with two loader warps each keep four streams going per SM.
+int env_int(const char* name, int dflt, int lo, int hi) {
+  const char* e = std::getenv(name);
+  if (e == nullptr) return dflt;
+  const int v = std::atoi(e);
+  return (v < lo || v > hi) ? dflt : v;
+}
+int ctas_per_sm() {
+  static const int v = env_int("SPENSE_CTAS_PER_SM", 2, 1, 2);
+  return v;
+}
+int producers() {
+  static const int v = env_int("SPENSE_PRODUCERS", 2, 1, 2);
+  return v;
+}
+int bulk_split() {
+  static const int v = [] {
+    const int x = env_int("SPENSE_BULK_SPLIT", 1, 1, 4);
+    return x == 3 ? 1 : x;
+  }();
+  return v;
+}
+
+// Checks that `count` handles can share one launch (same device, K, Kd and
+// dense column set) and plans it for M tokens on a device with `sms` SMs.
+spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, int sms, GemmPlan* out) {
+  if (hs == nullptr || count < 1 || count > kMaxGroup)
+    return fail(SPENSE_ERR_ARG, "a launch takes 1 to %d packed weights, got %d", kMaxGroup, count);
+  if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
+  const spense_packed* h0 = hs[0];
+  if (h0 == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
+  long long n_tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    const spense_packed* h = hs[i];
+    if (h == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
+    if (h->device != h0->device || h->K != h0->K || h->Kd != h0->Kd || h->perm_host != h0->perm_host)
+      return fail(SPENSE_ERR_ARG,
+                  "packed weights sharing a launch need the same device, K, Kd and dense column set");
+    n_tiles += h->n_tiles;
+  }
   GemmPlan pl{};
   pl.npad = M > kMaxTokenTile ? kMaxTokenTile : static_cast<int>(round_up(static_cast<size_t>(M), 16));
+  pl.box_rows = static_cast<int>(M > kMaxTokenTile ? kMaxTokenTile : M);
   pl.m_tiles = static_cast<int>((M + kMaxTokenTile - 1) / kMaxTokenTile);
-  pl.n_tiles = h->n_tiles;
+  pl.nsb = h0->nsb;
+  pl.ndb = h0->ndb;
+  const long long nblk = pl.nsb + pl.ndb;
+  if (n_tiles * pl.m_tiles * nblk >= (1ll << 31))
+    return fail(SPENSE_ERR_SHAPE, "too many blocks for one launch (%lld)", n_tiles * pl.m_tiles * nblk);
+  pl.n_tiles = static_cast<int>(n_tiles);
   pl.tiles = pl.n_tiles * pl.m_tiles;
-  pl.nsb = h->nsb;
-  pl.ndb = h->ndb;
   pl.tile_cost = kCostSparse * pl.nsb + kCostDense * pl.ndb;
   pl.total_cost = static_cast<long long>(pl.tiles) * pl.tile_cost;
   // Each CTA gets at least min_cta_weight() units of streamed bytes (never less
   // than one maximal block, so no CTA owns an empty range): small matrices are
   // split across fewer CTAs, which keeps the number of partials per tile low.
   long long grid = pl.total_cost / std::max<long long>(kCostSparse, min_cta_weight());
-  grid = std::max<long long>(1, std::min<long long>(grid, sms));
-  pl.grid = static_cast<int>(grid);
+  // Two CTAs per SM (two independent copy streams) when the token tile fits
+  // in half the shared and tensor memory; otherwise one.
+  pl.bulk_split = bulk_split();
+  pl.producers = producers();
   pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.nsb > 0 ? 256u : 128u);
   pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.nsb > 0 ? kMetaBlockBytes : 0);
   const uint32_t reserve = 1024 + 512;  // alignment slack + barriers
-  pl.stages = static_cast<int>(std::min<uint32_t>(kMaxStages, (gemm_max_smem() - reserve) / pl.stage_bytes));
-  pl.nacc = (2 * pl.npad + 16 <= 512) ? 2 : 1;
-  uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(pl.nacc * pl.npad + 16)) cols <<= 1;
-  pl.tmem_cols = cols;
+  for (int cps = ctas_per_sm(); cps >= 1; --cps) {
+    const uint32_t smem_budget = gemm_max_smem() / cps - (cps > 1 ? 1024u : 0u);
+    const uint32_t tmem_budget = 512u / cps;
+    const int stages = static_cast<int>(std::min<uint32_t>(kMaxStages, (smem_budget - reserve) / pl.stage_bytes));
+    const int nacc = (2u * pl.npad + 16u <= tmem_budget) ? 2 : 1;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(nacc * pl.npad + 16)) cols <<= 1;
+    if ((stages < 2 || cols > tmem_budget) && cps > 1) continue;
+    pl.ctas_per_sm = cps;
+    pl.stages = stages;
+    pl.nacc = nacc;
+    pl.tmem_cols = cols;
+    break;
+  }
+  grid = std::max<long long>(1, std::min<long long>(std::min<long long>(grid, static_cast<long long>(sms) * pl.ctas_per_sm), kMaxGrid));
+  pl.grid = static_cast<int>(grid);
+  // CTA g takes the blocks whose start weight falls in [g T / G, (g+1) T / G).
+  for (int g = 0; g <= pl.grid; ++g) {
+    const long long c = (static_cast<long long>(g) * pl.total_cost + pl.grid - 1) / pl.grid;
+    const long long t = c / pl.tile_cost;
+    const long long r = c - t * pl.tile_cost;
+    const long long sp = static_cast<long long>(kCostSparse) * pl.nsb;
+    const long long j = r <= sp ? (r + kCostSparse - 1) / kCostSparse : pl.nsb + (r - sp + kCostDense - 1) / kCostDense;
+    pl.cta_start[g] = static_cast<int>(t * nblk + j);
+  }
   pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
 
+  int64_t n_sum = 0;
+  for (int i = 0; i < count; ++i) n_sum += hs[i]->N;
   WorkspaceLayout& w = pl.ws;
   size_t off = 256;  // header: status word
   w.counters_off = off;
@@ -157,48 +228,53 @@ GemmPlan make_plan(const spense_packed* h, int64_t M, int sms) {
   w.partials_bytes = static_cast<size_t>(pl.grid) * 2 * pl.npad * kTileRows * 4;
   off += w.partials_bytes;
   w.xg_off = off;
-  w.xg_bytes = h->perm ? round_up(static_cast<size_t>(M * h->K), 256) : 0;
+  w.xg_bytes = h0->perm ? round_up(static_cast<size_t>(M * h0->K), 256) : 0;
   off += w.xg_bytes;
   w.total_device = off;
   w.stage_x_off = off;
-  off += round_up(static_cast<size_t>(M * h->K), 256);
+  off += round_up(static_cast<size_t>(M * h0->K), 256);
   w.stage_sx_off = off;
   off += round_up(static_cast<size_t>(M) * 4, 256);
   w.stage_y_off = off;
-  off += round_up(static_cast<size_t>(M * h->N) * 2, 256);
+  off += round_up(static_cast<size_t>(M * n_sum) * 2, 256);
   w.total_host = off;
-  return pl;
-}
-
-spense_status check_gemm_args(const spense_packed* Wp, int64_t M, void* workspace, int* dev,
-                              DeviceInfo* info) {
-  if (Wp == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
-  if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
-  if (workspace == nullptr) return fail(SPENSE_ERR_WORKSPACE, "workspace is NULL");
-  if (!aligned(workspace, 256)) return fail(SPENSE_ERR_ALIGN, "workspace is not 256-byte aligned");
-  spense_status st = current_device(dev, info);
-  if (st != SPENSE_OK) return st;
-  if (*dev != Wp->device)
-    return fail(SPENSE_ERR_ARG, "handle was packed on device %d, current device is %d", Wp->device, *dev);
+  *out = pl;
   return SPENSE_OK;
 }
 
-// Enqueue the GEMM on device buffers (arguments already validated).
-spense_status run_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale, int64_t M,
-                       uint16_t* Y, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream) {
+// Validates the call-level arguments shared by the GEMM entry points.
+spense_status check_gemm_args(const spense_packed* const* hs, int count, int64_t M, void* workspace,
+                              DeviceInfo* info) {
+  if (hs == nullptr || count < 1 || count > kMaxGroup || hs[0] == nullptr)
+    return fail(SPENSE_ERR_ARG, "Wp is NULL");
+  if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
+  if (workspace == nullptr) return fail(SPENSE_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(workspace, 256)) return fail(SPENSE_ERR_ALIGN, "workspace is not 256-byte aligned");
+  int dev = 0;
+  spense_status st = current_device(&dev, info);
+  if (st != SPENSE_OK) return st;
+  if (dev != hs[0]->device)
+    return fail(SPENSE_ERR_ARG, "handle was packed on device %d, current device is %d", hs[0]->device, dev);
+  return SPENSE_OK;
+}
+
+// Enqueue one launch over `count` packed weights sharing X (arguments validated).
+spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t* X, const float* x_scale,
+                       int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream) {
+  const spense_packed* h0 = hs[0];
   const uint8_t* xsrc = X;
-  if (Wp->perm != nullptr) {
+  if (h0->perm != nullptr) {
     uint8_t* xg = ws + pl.ws.xg_off;
-    cudaError_t e = launch_gather(X, Wp->perm, M, Wp->K, xg, stream);
+    cudaError_t e = launch_gather(X, h0->perm, M, h0->K, xg, stream);
     if (e != cudaSuccess) return cuda_fail(e, "gather launch");
     xsrc = xg;
   }
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return fail(SPENSE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
   CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(Wp->K), static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(Wp->K)};
-  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(pl.npad)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(h0->K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(h0->K)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(pl.box_rows)};
   const cuuint32_t estr[2] = {1u, 1u};
   CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(xsrc), dims, strides,
                       box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -206,32 +282,41 @@ spense_status run_gemm(const spense_packed* Wp, const uint8_t* X, const float* x
   if (r != CUDA_SUCCESS) return fail(SPENSE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
 
   GemmParams p{};
-  p.vs_t = Wp->vs_t;
-  p.e_t = Wp->e_t;
-  p.wd_t = Wp->wd_t;
-  p.s_w = Wp->s_w;
+  int tile_begin = 0;
+  for (int i = 0; i < count; ++i) {
+    GemmMember& m = p.mem[i];
+    m.vs_t = hs[i]->vs_t;
+    m.e_t = hs[i]->e_t;
+    m.wd_t = hs[i]->wd_t;
+    m.s_w = hs[i]->s_w;
+    m.y = Ys[i];
+    m.N = static_cast<int>(hs[i]->N);
+    m.tile_begin = tile_begin;
+    tile_begin += hs[i]->n_tiles;
+  }
+  p.n_members = count;
   p.s_x = x_scale;
-  p.y = Y;
   p.partials = reinterpret_cast<float*>(ws + pl.ws.partials_off);
   p.counters = reinterpret_cast<unsigned int*>(ws + pl.ws.counters_off);
   p.status = reinterpret_cast<unsigned int*>(ws);
-  p.N = static_cast<int>(Wp->N);
   p.M = static_cast<int>(M);
-  p.Ks = static_cast<int>(Wp->Ks);
-  p.Kd = static_cast<int>(Wp->Kd);
+  p.Ks = static_cast<int>(h0->Ks);
+  p.Kd = static_cast<int>(h0->Kd);
   p.n_tiles = pl.n_tiles;
   p.m_tiles = pl.m_tiles;
   p.nsb = pl.nsb;
   p.ndb = pl.ndb;
   p.npad = pl.npad;
+  p.box_rows = pl.box_rows;
   p.grid = pl.grid;
   p.stages = pl.stages;
   p.nacc = pl.nacc;
-  p.tile_cost = pl.tile_cost;
-  p.total_cost = pl.total_cost;
   p.stage_bytes = pl.stage_bytes;
   p.b_bytes = pl.b_bytes;
   p.tmem_cols = pl.tmem_cols;
+  std::memcpy(p.cta_start, pl.cta_start, sizeof(int) * (pl.grid + 1));
+  p.bulk_split = pl.bulk_split;
+  p.producers = pl.producers;
   cudaError_t e = launch_gemm(map, p, pl.smem_bytes, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return SPENSE_OK;
@@ -341,6 +426,7 @@ spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int
     for (int64_t j = 0; j < Kd; ++j) perm.push_back(dense_idx[j]);
     e = cudaMemcpyAsync(h->perm, perm.data(), perm.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // `perm` is a host temporary
+    h->perm_host = perm;
   }
   if (e == cudaSuccess) e = cudaMemsetAsync(err_d, 0, sizeof(unsigned int), stream);
   if (e == cudaSuccess)
@@ -374,37 +460,58 @@ spense_status spense_free(spense_packed* Wp) {
 }
 
 size_t spense_gemm_workspace_size(const spense_packed* Wp, int64_t M) {
-  if (Wp == nullptr || M < 1 || M > 65535) return 0;
+  return spense_gemm_grouped_workspace_size(&Wp, 1, M);
+}
+
+size_t spense_gemm_grouped_workspace_size(const spense_packed* const* Wps, int count, int64_t M) {
   int dev = 0;
   DeviceInfo info;
   if (current_device(&dev, &info) != SPENSE_OK) return 0;
-  return make_plan(Wp, M, info.sms).ws.total_device;
+  GemmPlan pl;
+  if (make_plan(Wps, count, M, info.sms, &pl) != SPENSE_OK) return 0;
+  return pl.ws.total_device;
 }
 
 size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M) {
-  if (Wp == nullptr || M < 1 || M > 65535) return 0;
   int dev = 0;
   DeviceInfo info;
   if (current_device(&dev, &info) != SPENSE_OK) return 0;
-  return make_plan(Wp, M, info.sms).ws.total_host;
+  GemmPlan pl;
+  if (make_plan(&Wp, 1, M, info.sms, &pl) != SPENSE_OK) return 0;
+  return pl.ws.total_host;
+}
+
+spense_status spense_gemm_grouped(const spense_packed* const* Wps, int count, const uint8_t* X,
+                                  const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
+                                  size_t workspace_bytes, void* stream_v) {
+  if (X == nullptr || x_scale == nullptr || Ys == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
+  if (!aligned(X, 16) || !aligned(x_scale, 4))
+    return fail(SPENSE_ERR_ALIGN, "X must be 16-byte aligned, x_scale 4-byte aligned");
+  if (count >= 1 && count <= kMaxGroup) {
+    for (int i = 0; i < count; ++i) {
+      if (Ys[i] == nullptr) return fail(SPENSE_ERR_ARG, "Y[%d] is NULL", i);
+      if (!aligned(Ys[i], 16)) return fail(SPENSE_ERR_ALIGN, "Y[%d] must be 16-byte aligned", i);
+    }
+  }
+  DeviceInfo info;
+  spense_status st = check_gemm_args(Wps, count, M, workspace, &info);
+  if (st != SPENSE_OK) return st;
+  GemmPlan pl;
+  st = make_plan(Wps, count, M, info.sms, &pl);
+  if (st != SPENSE_OK) return st;
+  if (workspace_bytes < pl.ws.total_device)
+    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                pl.ws.total_device);
+  st = run_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
+                static_cast<cudaStream_t>(stream_v));
+  return st == SPENSE_OK ? ok() : st;
 }
 
 spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale, int64_t M,
                           uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream_v) {
-  if (X == nullptr || x_scale == nullptr || Y == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
-  if (!aligned(X, 16) || !aligned(Y, 16) || !aligned(x_scale, 4))
-    return fail(SPENSE_ERR_ALIGN, "X and Y must be 16-byte aligned, x_scale 4-byte aligned");
-  int dev = 0;
-  DeviceInfo info;
-  spense_status st = check_gemm_args(Wp, M, workspace, &dev, &info);
-  if (st != SPENSE_OK) return st;
-  const GemmPlan pl = make_plan(Wp, M, info.sms);
-  if (workspace_bytes < pl.ws.total_device)
-    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
-                pl.ws.total_device);
-  st = run_gemm(Wp, X, x_scale, M, Y, static_cast<uint8_t*>(workspace), pl,
-                static_cast<cudaStream_t>(stream_v));
-  return st == SPENSE_OK ? ok() : st;
+  if (Y == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
+  if (X != nullptr && !aligned(X, 16)) return fail(SPENSE_ERR_ALIGN, "X and Y must be 16-byte aligned");
+  return spense_gemm_grouped(&Wp, 1, X, x_scale, M, &Y, workspace, workspace_bytes, stream_v);
 }
 
 spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host, const float* x_scale_host,
@@ -412,11 +519,12 @@ spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host, c
                                void* stream_v) {
   if (X_host == nullptr || x_scale_host == nullptr || Y_host == nullptr)
     return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
-  int dev = 0;
   DeviceInfo info;
-  spense_status st = check_gemm_args(Wp, M, workspace, &dev, &info);
+  spense_status st = check_gemm_args(&Wp, 1, M, workspace, &info);
   if (st != SPENSE_OK) return st;
-  const GemmPlan pl = make_plan(Wp, M, info.sms);
+  GemmPlan pl;
+  st = make_plan(&Wp, 1, M, info.sms, &pl);
+  if (st != SPENSE_OK) return st;
   if (workspace_bytes < pl.ws.total_host)
     return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
                 pl.ws.total_host);
@@ -429,7 +537,7 @@ spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host, c
   if (e == cudaSuccess)
     e = cudaMemcpyAsync(sxd, x_scale_host, static_cast<size_t>(M) * 4, cudaMemcpyHostToDevice, stream);
   if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-  st = run_gemm(Wp, xd, sxd, M, yd, ws, pl, stream);
+  st = run_gemm(&Wp, 1, xd, sxd, M, &yd, ws, pl, stream);
   if (st != SPENSE_OK) return st;
   e = cudaMemcpyAsync(Y_host, yd, static_cast<size_t>(M * Wp->N) * 2, cudaMemcpyDeviceToHost, stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
@@ -488,7 +596,9 @@ spense_status spense_gemm_noalloc(const spense_packed* Wp, const uint8_t* X, con
   if (st != SPENSE_OK) return st;
   if (dev != Wp->device)
     return fail(SPENSE_ERR_ARG, "handle was packed on device %d, current device is %d", Wp->device, dev);
-  const GemmPlan pl = make_plan(Wp, M, info.sms);
+  GemmPlan pl;
+  st = make_plan(&Wp, 1, M, info.sms, &pl);
+  if (st != SPENSE_OK) return st;
   if (pl.ws.total_device > SPENSE_NOALLOC_SCRATCH_BYTES)
     return fail(SPENSE_ERR_WORKSPACE,
                 "this GEMM needs %zu bytes of scratch; the built-in scratch holds %zu (use spense_gemm "
@@ -502,7 +612,7 @@ spense_status spense_gemm_noalloc(const spense_packed* Wp, const uint8_t* X, con
   // keeps whatever the previous call left in it.
   const cudaError_t e = cudaMemsetAsync(ws, 0, pl.ws.partials_off, stream);
   if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
-  st = run_gemm(Wp, X, x_scale, M, Y, ws, pl, stream);
+  st = run_gemm(&Wp, 1, X, x_scale, M, &Y, ws, pl, stream);
   return st == SPENSE_OK ? ok() : st;
 }
 

@@ -19,6 +19,7 @@ constexpr int kMaxTokenTile = 256;      // tokens per tile (MMA N upper bound)
 constexpr int kCostSparse = 5;          // HBM bytes of a sparse block in 4 KiB units (16 + 4 KiB)
 constexpr int kCostDense = 4;           // ... of a dense block (16 KiB)
 constexpr int kGemmThreads = 192;       // warp 0 loads, warp 1 issues MMAs, warps 2-5 epilogue
+constexpr int kGemmThreadsMax = 224;    // plus warp 6 as a second loader
 constexpr int kMaxStages = 12;
 
 // Workspace layout: [header 256 B][counters][partials][gathered X][host staging]
@@ -31,10 +32,14 @@ struct WorkspaceLayout {
   size_t total_host;    // bytes for spense_gemm_host
 };
 
+constexpr int kMaxGroup = 4;    // weight matrices sharing one activation tensor in one launch
+constexpr int kMaxGrid = 320;   // CTAs per launch (up to two per SM)
+
 struct GemmPlan {
   int npad;        // MMA N (tokens per tile, multiple of 16)
+  int box_rows;    // activation rows one TMA box loads (<= npad)
   int m_tiles;
-  int n_tiles;
+  int n_tiles;     // row tiles over all group members
   int tiles;       // n_tiles * m_tiles
   int nsb, ndb;    // sparse / dense blocks per tile
   int tile_cost;   // kCostSparse * nsb + kCostDense * ndb
@@ -46,26 +51,40 @@ struct GemmPlan {
   int nacc;          // accumulator buffers in tensor memory
   uint32_t tmem_cols;
   uint32_t smem_bytes;
+  int ctas_per_sm;
+  int bulk_split;
+  int producers;
+  int cta_start[kMaxGrid + 1];  // first linear block of each CTA; [grid] = total blocks
   WorkspaceLayout ws;
 };
 
-struct GemmParams {
+// One weight matrix of a launch: its packed blocks, scales, output and the
+// first global row tile it occupies.
+struct GemmMember {
   const uint8_t* vs_t;
   const uint8_t* e_t;
   const uint8_t* wd_t;
   const float* s_w;
-  const float* s_x;
   uint16_t* y;
+  int N;
+  int tile_begin;
+};
+
+struct GemmParams {
+  GemmMember mem[kMaxGroup];
+  int n_members;
+  const float* s_x;
   float* partials;
   unsigned int* counters;
   unsigned int* status;
-  int N, M, Ks, Kd;
+  int M, Ks, Kd;
   int n_tiles, m_tiles, nsb, ndb;
-  int npad, grid, stages, nacc;
-  int tile_cost;
-  long long total_cost;
+  int npad, box_rows, grid, stages, nacc;
   uint32_t stage_bytes, b_bytes;
   uint32_t tmem_cols;
+  int cta_start[kMaxGrid + 1];
+  int bulk_split;  // weight block copied as this many bulk copies (1, 2 or 4)
+  int producers;   // loader warps (1 or 2)
 };
 
 // Kernels (defined in the .cu files).

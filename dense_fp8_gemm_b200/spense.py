@@ -28,7 +28,9 @@ SYMBOLS = (
     "spense_pack", "spense_gemm", "spense_gemm_workspace_size", "spense_gemm_host",
     "spense_gemm_host_workspace_size", "spense_free", "spense_get_info",
     "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
+    "spense_gemm_grouped", "spense_gemm_grouped_workspace_size",
 )
+MAX_GROUP = 4
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
@@ -71,10 +73,13 @@ def lib() -> ctypes.CDLL:
     L.spense_get_info.argtypes = [P, ctypes.POINTER(PackedInfo)]
     L.spense_workspace_status.argtypes = [P, P, ctypes.POINTER(U32)]
     L.spense_gemm_noalloc.argtypes = [P, P, P, I64, P, P]
+    L.spense_gemm_grouped.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ, P]
+    L.spense_gemm_grouped_workspace_size.argtypes = [ctypes.POINTER(P), ctypes.c_int, I64]
+    L.spense_gemm_grouped_workspace_size.restype = SZ
     L.spense_last_error.restype = ctypes.c_char_p
     L.spense_version.restype = ctypes.c_char_p
     for name in ("spense_pack", "spense_gemm", "spense_gemm_host", "spense_free", "spense_get_info",
-                 "spense_workspace_status", "spense_gemm_noalloc"):
+                 "spense_workspace_status", "spense_gemm_noalloc", "spense_gemm_grouped"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -244,6 +249,40 @@ def gemm_host(pw: PackedWeight, X_host: torch.Tensor, x_scale_host: torch.Tensor
                                   _stream(stream))
     _check(code, "spense_gemm_host")
     return Y_host
+
+
+def _handles(pws):
+    arr = (ctypes.c_void_p * len(pws))()
+    for i, pw in enumerate(pws):
+        arr[i] = pw.handle.value
+    return arr
+
+
+def grouped_workspace_size(pws, M: int) -> int:
+    n = lib().spense_gemm_grouped_workspace_size(_handles(pws), len(pws), M)
+    if n == 0:
+        _check(1, "spense_gemm_grouped_workspace_size")
+    return int(n)
+
+
+def gemm_grouped(pws, X: torch.Tensor, x_scale: torch.Tensor, Ys=None, workspace: torch.Tensor | None = None,
+                 stream=None):
+    """spense_gemm_grouped: one launch over several packed weights sharing X
+    (same K, Kd and dense column set). Returns the list of outputs."""
+    M = X.shape[0]
+    if Ys is None:
+        Ys = [torch.empty((M, pw.N), dtype=torch.bfloat16, device=X.device) for pw in pws]
+    if workspace is None:
+        workspace = new_workspace(grouped_workspace_size(pws, M), X.device)
+    yarr = (ctypes.c_void_p * len(pws))()
+    for i, Y in enumerate(Ys):
+        yarr[i] = _dev_ptr(Y, torch.bfloat16, f"Y[{i}]").value
+    code = lib().spense_gemm_grouped(_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"),
+                                     _dev_ptr(x_scale, torch.float32, "x_scale"), M, yarr,
+                                     _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                     _stream(stream))
+    _check(code, "spense_gemm_grouped")
+    return Ys
 
 
 def gemm_noalloc(pw: PackedWeight, X: torch.Tensor, x_scale: torch.Tensor, Y: torch.Tensor,

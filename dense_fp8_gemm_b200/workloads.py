@@ -110,3 +110,16 @@ def useful_flops(N: int, K: int, Kd: int, M: int) -> int:
     """2 * M * N * (nonzero weights per row)."""
     Ks = K - Kd
     return 2 * M * N * (Ks // 2 + Kd)
+
+
+def group_algorithmic_bytes(members, M: int) -> int:
+    """Algorithmic bytes of one launch over weights (N_i, K, Kd) sharing one
+    activation tensor: every member's packed weights, scales and output, and the
+    shared activations once."""
+    K = members[0][1]
+    total = M * K + 4 * M
+    for N, k, Kd in members:
+        assert k == K
+        total += weight_bytes(N, K, Kd) + 4 * N + 2 * M * N
+    return total
+

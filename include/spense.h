@@ -141,6 +141,25 @@ SPENSE_API spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, 
 SPENSE_API size_t spense_gemm_workspace_size(const spense_packed* Wp, int64_t M);
 
 /*
+ * spense_gemm_grouped — one launch over `count` (1..4) packed weights that share
+ * the activations X: Ys[i] [M][N_i] = X * Wp_i^T with scales. The weights must
+ * have been packed on the same device with the same K, Kd and dense column set
+ * (for example the q, k and v projections of one layer, or gate and up). Their
+ * row tiles are streamed as one sequence, so small matrices share the SMs and
+ * the launch cost instead of each paying for its own launch. This is a fusion
+ * of independent GEMMs over one input; each output is exactly what spense_gemm
+ * gives for that weight.
+ *   workspace  at least spense_gemm_grouped_workspace_size(Wps, count, M) bytes,
+ *              with the same rules as for spense_gemm.
+ * Errors: as spense_gemm, plus ARG when the weights cannot share a launch.
+ */
+SPENSE_API spense_status spense_gemm_grouped(const spense_packed* const* Wps, int count, const uint8_t* X,
+                                             const float* x_scale, int64_t M, uint16_t* const* Ys,
+                                             void* workspace, size_t workspace_bytes, void* stream);
+
+SPENSE_API size_t spense_gemm_grouped_workspace_size(const spense_packed* const* Wps, int count, int64_t M);
+
+/*
  * spense_gemm_host — the same GEMM on HOST buffers: copies X [M][K] and
  * x_scale [M] from host memory into the workspace, runs spense_gemm, copies Y
  * [M][N] back to host memory and synchronizes `stream` before returning.

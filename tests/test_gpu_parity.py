@@ -225,3 +225,57 @@ def test_spensegpt_plus_sweep(df):
 @pytest.mark.parametrize("i", range(6))
 def test_chain36b_layer(i):
     _check_workload_shape(workloads.CHAIN36B, i, workloads.CHAIN36B.batches)
+
+
+# --------------------------------------------------------------------------- grouped launches
+
+
+@pytest.mark.parametrize("M,Ns,K,Kd,scattered", [
+    (16, (384, 128, 128), 1024, 256, False),
+    (5, (200, 72, 330), 640, 160, False),       # ragged row counts in every member
+    (40, (256, 256), 768, 256, True),            # shared SpenseGPT+ dense set
+    (300, (128, 256, 128, 128), 512, 128, False),
+])
+def test_grouped_matches_oracle(M, Ns, K, Kd, scattered):
+    X, s_x = synth.quantize_rows(synth.normal(55 + M, 1, (M, K), 1.0))
+    idx = synth.scored_dense_idx(55, 3, K, Kd) if scattered else None
+    pws, refs = [], []
+    for i, N in enumerate(Ns):
+        W, s_w = synth.quantize_rows(synth.normal(55 + M, 10 + i, (N, K), 0.02))
+        keep = oracle.pack(W, dense_idx=idx, Kd=Kd)["keep"]
+        refs.append(oracle.gemm(X, s_x, W, s_w, keep=keep))
+        pws.append(spense.pack(_dev(W), _dev(s_w), Kd=Kd, dense_idx=idx))
+    ws = spense.new_workspace(spense.grouped_workspace_size(pws, M))
+    Ys = spense.gemm_grouped(pws, _dev(X), _dev(s_x), workspace=ws)
+    torch.cuda.synchronize()
+    assert spense.workspace_status(ws) == 0
+    for i, (Y, (yref, bound)) in enumerate(zip(Ys, refs)):
+        _assert_close(Y, yref, bound, f"member {i}")
+
+
+@pytest.mark.parametrize("M", [1, 16])
+def test_grouped_attn32b_qkv(M):
+    wl = workloads.ATTN32B
+    X, s_x = workloads.make_activations(wl, 0, M)
+    pws, checks = [], []
+    for i in range(3):  # q, k, v share the input of the layer
+        w = workloads.make_weight(wl, i)
+        rows = _sample_rows(w.N, seed=i)
+        keep = oracle.pack(w.W[rows], Kd=w.Kd)["keep"]
+        checks.append((rows, oracle.gemm(X, s_x, w.W[rows], w.s_w[rows], keep=keep)))
+        pws.append(spense.pack(_dev(w.W), _dev(w.s_w), Kd=w.Kd))
+    Ys = spense.gemm_grouped(pws, _dev(X), _dev(s_x))
+    torch.cuda.synchronize()
+    for i, (Y, (rows, (yref, bound))) in enumerate(zip(Ys, checks)):
+        _assert_close(Y[:, torch.from_numpy(rows).cuda()], yref, bound, f"qkv member {i} M={M}")
+
+
+def test_grouped_rejects_mismatched_layouts():
+    K = 512
+    W, s_w = synth.quantize_rows(synth.normal(77, 1, (128, K), 0.02))
+    a = spense.pack(_dev(W), _dev(s_w), Kd=128)
+    b = spense.pack(_dev(W), _dev(s_w), Kd=256)
+    X, s_x = synth.quantize_rows(synth.normal(77, 2, (4, K), 1.0))
+    with pytest.raises(spense.SpenseError) as ei:
+        spense.gemm_grouped([a, b], _dev(X), _dev(s_x), workspace=spense.new_workspace(1 << 20))
+    assert ei.value.code == 1
