@@ -53,6 +53,7 @@ struct alignas(8) Barriers {
   uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t peer_done;  // cluster mode: one arrival per peer CTA whose partial is ready
   uint32_t tmem_base;
   int abort_flag;
   int fix_flag;
@@ -65,6 +66,24 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, unsigned
   uint32_t it = 0;
   while (true) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
+    if ((++it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        atomicOr(status, code);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait with acquire at cluster scope (for arrivals from peer CTAs).
+__device__ __forceinline__ bool wait_bar_cluster(uint32_t bar, uint32_t parity, unsigned int* status,
+                                                 unsigned int code, volatile int* abort_flag) {
+  const uint64_t t0 = ptx::globaltimer();
+  uint32_t it = 0;
+  while (true) {
+    if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
     if ((++it & 63u) == 0) {
       if (*abort_flag) return false;
       if (ptx::globaltimer() - t0 > kWaitLimitNs) {
@@ -188,6 +207,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
       ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), 128);
     }
+    ptx::mbar_init(ptx::smem_addr(&bars->peer_done), p.cluster > 1 ? p.cluster - 1 : 1);
     bars->abort_flag = 0;
     bars->fix_flag = 0;
     ptx::fence_mbar_init();
@@ -199,6 +219,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   }
   ptx::tc_fence_before();
   __syncthreads();
+  if (p.cluster > 1) ptx::cluster_sync();  // peers' barriers are initialised before any remote arrive
   ptx::tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
   volatile int* abort_flag = &bars->abort_flag;
@@ -342,15 +363,11 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
-    for (int u = 0; u < units.count; ++u) {
-      int t, j0, j1;
-      units.get(u, t, j0, j1);
-      const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
-      const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
-      const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
-                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
-      ptx::tc_fence_after();
+
+    // Sum the contributors' partials of tile t in CTA order and store Y. Every
+    // contributor after g_lo starts inside tile t, so its partial is in slot
+    // 0; g_lo uses slot 1 when its range started in an earlier tile.
+    auto finish_tile = [&](int t) {
       const int n_tile = t / p.m_tiles;
       const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
@@ -358,57 +375,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       const int n = (n_tile - mb.tile_begin) * kTileRows + row;
       const bool row_ok = n < mb.N;
       const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
-      const bool whole = (j0 == 0 && j1 == nblk);
-      const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
-      // Partials are stored [CTA][slot][row][npad]: slot 0 for the tile holding the
-      // CTA's first block, slot 1 for the tile holding its last block.
-      float* part = nullptr;
-      if (!whole) {
-        const int slot = (b0 >= t * nblk) ? 0 : 1;
-        part = p.partials + (static_cast<size_t>(g) * 2 + slot) * slot_elems + static_cast<size_t>(row) * p.npad;
-      }
-      for (int c0 = 0; c0 < m_valid; c0 += 16) {
-        uint32_t v[16];
-        ptx::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), v);
-        ptx::tmem_ld_wait();
-        if (whole) {
-          if (row_ok) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int m = c0 + i;
-              if (m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] =
-                    to_bf16_bits(__uint_as_float(v[i]) * sw * __ldg(p.s_x + m0 + m));
-            }
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(part + c0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (c0 + 4 * q < m_valid)
-              __stcg(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
-        }
-      }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
-      if (whole) continue;
-
-      // Publish this CTA's partial: the named barrier orders the 128 threads'
-      // stores before thread 0's release-acquire ticket at GPU scope.
-      ptx::named_bar_sync(1, 128);
       const int g_lo = block_owner(p, t * nblk);
       const int g_hi = block_owner(p, t * nblk + nblk - 1);
-      if (et == 0) {
-        const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
-        bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
-      }
-      ptx::named_bar_sync(1, 128);
-      if (!*reinterpret_cast<volatile int*>(&bars->fix_flag)) continue;
-
-      // Last to arrive: sum the contributors' partials in CTA order. Every
-      // contributor after g_lo starts inside tile t, so its partial is in slot
-      // 0; g_lo uses slot 1 when its range started in an earlier tile.
       const int lo_slot = (p.cta_start[g_lo] >= t * nblk) ? 0 : 1;
       const float* lo_part =
           p.partials + (static_cast<size_t>(g_lo) * 2 + lo_slot) * slot_elems + static_cast<size_t>(row) * p.npad;
@@ -462,12 +430,164 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         }
       }
       if (et == 0) p.counters[t] = 0u;  // re-arm for the next launch (ordered by the kernel boundary)
+    };
+
+    // Tiles this CTA must finish. Their fix-ups wait until this CTA has
+    // published the partials of all its shared tiles (which come first in the
+    // processing order), so no other CTA's fix-up waits behind this one's.
+    int pending[2];
+    int npending = 0;
+    if (p.cluster > 1 && units.count == 1) {
+      // Cluster split: the S CTAs of a cluster hold consecutive K ranges of one
+      // tile. Peers leave their fp32 partial in their own (now idle) stage
+      // memory and signal rank 0, which adds them in rank order through
+      // distributed shared memory and stores Y.
+      int t, j0, j1;
+      units.get(0, t, j0, j1);
+      const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[0]), 0, p.status,
+                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
+      if (__all_sync(0xffffffffu, got)) {
+        ptx::tc_fence_after();
+        const int n_tile = t / p.m_tiles;
+        const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+        const GemmMember& mb = p.mem[member_of(p, n_tile)];
+        const int m_valid = min(p.npad, p.M - m0);
+        const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+        const bool row_ok = n < mb.N;
+        const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
+        const uint32_t rank = ptx::cluster_ctarank();
+        const uint32_t part_s = smem_base + static_cast<uint32_t>(row * p.npad) * 4u;
+        if (rank != 0) {
+          for (int c0 = 0; c0 < m_valid; c0 += 16) {
+            uint32_t v[16];
+            ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c0), v);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              ptx::st_smem_v4(part_s + static_cast<uint32_t>(c0 + 4 * q) * 4u,
+                              make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+          }
+          ptx::tc_fence_before();
+          ptx::named_bar_sync(1, 128);
+          if (et == 0) ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_addr(&bars->peer_done), 0));
+        } else if (wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status, SPENSE_DEVICE_TIMEOUT_EPILOGUE,
+                                    abort_flag)) {
+          for (int c0 = 0; c0 < m_valid; c0 += 16) {
+            uint32_t v[16];
+            ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c0), v);
+            ptx::tmem_ld_wait();
+            float a[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
+            for (int r = 1; r < p.cluster; ++r) {
+              const uint32_t src = ptx::mapa(part_s + static_cast<uint32_t>(c0) * 4u, static_cast<uint32_t>(r));
+              float4 b[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) b[q] = ptx::ld_dsmem_v4(src + 16u * q);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                a[4 * q] += b[q].x;
+                a[4 * q + 1] += b[q].y;
+                a[4 * q + 2] += b[q].z;
+                a[4 * q + 3] += b[q].w;
+              }
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const int m = c0 + i;
+                if (m < m_valid)
+                  mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(a[i] * sw * __ldg(p.s_x + m0 + m));
+              }
+            }
+          }
+          ptx::tc_fence_before();
+        }
+      }
+    }
+    for (int u = 0; p.cluster <= 1 && u < units.count; ++u) {
+      int t, j0, j1;
+      units.get(u, t, j0, j1);
+      const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
+      const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
+      const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
+                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
+      ptx::tc_fence_after();
+      const int n_tile = t / p.m_tiles;
+      const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      const GemmMember& mb = p.mem[member_of(p, n_tile)];
+      const int m_valid = min(p.npad, p.M - m0);
+      const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+      const bool row_ok = n < mb.N;
+      const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
+      const bool whole = (j0 == 0 && j1 == nblk);
+      const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
+      // Partials are stored [CTA][slot][row][npad]: slot 0 for the tile holding the
+      // CTA's first block, slot 1 for the tile holding its last block.
+      float* part = nullptr;
+      if (!whole) {
+        const int slot = (b0 >= t * nblk) ? 0 : 1;
+        part = p.partials + (static_cast<size_t>(g) * 2 + slot) * slot_elems + static_cast<size_t>(row) * p.npad;
+      }
+      for (int c0 = 0; c0 < m_valid; c0 += 16) {
+        uint32_t v[16];
+        ptx::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), v);
+        ptx::tmem_ld_wait();
+        if (whole) {
+          if (row_ok) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int m = c0 + i;
+              if (m < m_valid)
+                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] =
+                    to_bf16_bits(__uint_as_float(v[i]) * sw * __ldg(p.s_x + m0 + m));
+            }
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(part + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            if (c0 + 4 * q < m_valid)
+              __stcg(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
+      if (!whole) {
+        // Publish this CTA's partial: the named barrier orders the 128 threads'
+        // stores before thread 0's release-acquire ticket at GPU scope.
+        ptx::named_bar_sync(1, 128);
+        if (et == 0) {
+          const int g_lo = block_owner(p, t * nblk);
+          const int g_hi = block_owner(p, t * nblk + nblk - 1);
+          const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
+          bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
+        }
+        ptx::named_bar_sync(1, 128);
+        if (*reinterpret_cast<volatile int*>(&bars->fix_flag) && npending < 2) pending[npending++] = t;
+      }
+      // Shared tiles come first; once the next unit is whole (or none is left),
+      // every ticket of this CTA is out and the pending fix-ups can run.
+      bool next_whole = true;
+      if (u + 1 < units.count) {
+        int t2, a2, b2;
+        units.get(u + 1, t2, a2, b2);
+        next_whole = (a2 == 0 && b2 == nblk);
+      }
+      if (next_whole) {
+        for (int i = 0; i < npending; ++i) finish_tile(pending[i]);
+        npending = 0;
+      }
     }
   }
 
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
+  if (p.cluster > 1) ptx::cluster_sync();  // peers keep their shared memory until rank 0 has read it
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, p.tmem_cols);
@@ -477,6 +597,17 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
 }  // namespace
 
 uint32_t gemm_max_smem() { return 232448u; }
+
+// Clusters may share SMs (two CTAs per SM) rather than spread one CTA per SM.
+cudaClusterSchedulingPolicy cluster_policy() {
+  static const cudaClusterSchedulingPolicy v = [] {
+    const char* e = std::getenv("SPENSE_CLUSTER_POLICY");
+    if (e != nullptr && e[0] == 's') return cudaClusterSchedulingPolicySpread;
+    if (e != nullptr && e[0] == 'd') return cudaClusterSchedulingPolicyDefault;
+    return cudaClusterSchedulingPolicyLoadBalancing;
+  }();
+  return v;
+}
 
 cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t smem_bytes,
                         cudaStream_t stream) {
@@ -502,11 +633,17 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
   cfg.blockDim = dim3(kGemmThreads + 32 * (p.producers - 1));
   cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned int>(p.cluster > 1 ? p.cluster : 1);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  attr[2].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+  attr[2].val.clusterSchedulingPolicyPreference = cluster_policy();
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = p.cluster > 1 ? 3 : 2;
   return cudaLaunchKernelEx(&cfg, spense_gemm_kernel, tmap_x, p);
 }
 

@@ -141,6 +141,13 @@ int producers() {
   static const int v = env_int("SPENSE_PRODUCERS", 2, 1, 2);
   return v;
 }
+// SPENSE_CLUSTER: 0 = stream-K only, 1 = automatic (default), 2/4/8 = that
+// cluster size whenever it fits.
+int cluster_mode() {
+  static const int v = env_int("SPENSE_CLUSTER", 1, 0, 8);
+  return v;
+}
+
 int bulk_split() {
   static const int v = [] {
     const int x = env_int("SPENSE_BULK_SPLIT", 1, 1, 4);
@@ -204,19 +211,50 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     pl.tmem_cols = cols;
     break;
   }
-  grid = std::max<long long>(1, std::min<long long>(std::min<long long>(grid, static_cast<long long>(sms) * pl.ctas_per_sm), kMaxGrid));
-  pl.grid = static_cast<int>(grid);
-  // CTA g takes the blocks whose start weight falls in [g T / G, (g+1) T / G).
-  for (int g = 0; g <= pl.grid; ++g) {
-    const long long c = (static_cast<long long>(g) * pl.total_cost + pl.grid - 1) / pl.grid;
-    const long long t = c / pl.tile_cost;
-    const long long r = c - t * pl.tile_cost;
+  const long long slots = std::min<long long>(static_cast<long long>(sms) * pl.ctas_per_sm, kMaxGrid);
+  // First block of a tile whose start weight is >= c (c within one tile).
+  auto block_at = [&](long long c) {
     const long long sp = static_cast<long long>(kCostSparse) * pl.nsb;
-    const long long j = r <= sp ? (r + kCostSparse - 1) / kCostSparse : pl.nsb + (r - sp + kCostDense - 1) / kCostDense;
-    pl.cta_start[g] = static_cast<int>(t * nblk + j);
+    return c <= sp ? (c + kCostSparse - 1) / kCostSparse : pl.nsb + (c - sp + kCostDense - 1) / kCostDense;
+  };
+  // Few tiles (at most half the CTA slots): the CTAs of a cluster of S split
+  // each tile's K range by weight and reduce in shared memory; otherwise
+  // stream-K over all tiles with the global fix-up.
+  pl.cluster = 1;
+  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
+  const int mode = cluster_mode();
+  if (mode != 0 && pl.tiles * 2 <= slots && pl.npad <= 64) {
+    // Power-of-two cluster sizes (a grid of clusters of 7 did not fit in one
+    // wave); the cluster grid must fit the CTA slots and fill at least half of
+    // them, unless the GEMM is so small that fixed costs dominate anyway.
+    for (int S = 8; S >= 2; S >>= 1) {
+      if (mode > 1 && S != mode) continue;
+      if (pl.tiles * S > slots || S > pl.tile_cost / kCostSparse) continue;
+      const bool fills = pl.tiles * S * 2 >= slots;
+      const bool small = pl.total_cost < 40LL * slots;
+      if (mode > 1 || fills || small) {
+        pl.cluster = S;
+        break;
+      }
+    }
+  }
+  if (pl.cluster > 1) {
+    pl.grid = pl.tiles * pl.cluster;
+    for (int g = 0; g <= pl.grid; ++g) {
+      const long long t = g / pl.cluster, r = g % pl.cluster;
+      pl.cta_start[g] = static_cast<int>(t * nblk + block_at((r * pl.tile_cost + pl.cluster - 1) / pl.cluster));
+    }
+  } else {
+    grid = std::max<long long>(1, std::min<long long>(grid, slots));
+    pl.grid = static_cast<int>(grid);
+    // CTA g takes the blocks whose start weight falls in [g T / G, (g+1) T / G).
+    for (int g = 0; g <= pl.grid; ++g) {
+      const long long c = (static_cast<long long>(g) * pl.total_cost + pl.grid - 1) / pl.grid;
+      const long long t = c / pl.tile_cost;
+      pl.cta_start[g] = static_cast<int>(t * nblk + block_at(c - t * pl.tile_cost));
+    }
   }
   pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
-
   int64_t n_sum = 0;
   for (int i = 0; i < count; ++i) n_sum += hs[i]->N;
   WorkspaceLayout& w = pl.ws;
@@ -317,6 +355,7 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
   std::memcpy(p.cta_start, pl.cta_start, sizeof(int) * (pl.grid + 1));
   p.bulk_split = pl.bulk_split;
   p.producers = pl.producers;
+  p.cluster = pl.cluster;
   cudaError_t e = launch_gemm(map, p, pl.smem_bytes, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return SPENSE_OK;

@@ -54,6 +54,7 @@ struct GemmPlan {
   int ctas_per_sm;
   int bulk_split;
   int producers;
+  int cluster;
   int cta_start[kMaxGrid + 1];  // first linear block of each CTA; [grid] = total blocks
   WorkspaceLayout ws;
 };
@@ -85,6 +86,7 @@ struct GemmParams {
   int cta_start[kMaxGrid + 1];
   int bulk_split;  // weight block copied as this many bulk copies (1, 2 or 4)
   int producers;   // loader warps (1 or 2)
+  int cluster;     // > 1: CTAs of a cluster split one tile's K and reduce through shared memory
 };
 
 // Kernels (defined in the .cu files).
