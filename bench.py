@@ -63,6 +63,7 @@ def workload_config(args):
         "dense_columns": "tail (SpenseGPT)",
         "weights": "FP8 e4m3 N(0,0.02) per-channel absmax scales; X N(0,1) per-token scales; seed 1",
         "l2": f"{args.layers} weight sets rotated per step (inputs larger than L2)",
+        "graph": f"one CUDA graph per {args.layers} steps (the rotated layers back to back)",
     }
 
 
@@ -250,15 +251,12 @@ def run_reference(args):
 
 def run_spense(args):
     import torch
-    import torch.distributed as dist
 
-    from dense_fp8_gemm_b200 import spense, workloads
+    from dense_fp8_gemm_b200 import replicas, spense, workloads
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    ranks = replicas.from_env()
+    world, rank, local = ranks.world, ranks.rank, ranks.local
+    replicas.init(ranks, "nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
@@ -295,6 +293,18 @@ def run_spense(args):
             if events is not None:
                 events[gi][1].record(stream)
 
+    def capture_chain(layer_list):
+        """One graph over all layers in sequence (a decode step of the whole stack)."""
+        for L in layer_list:
+            launch_layer(L, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for L in layer_list:
+                launch_layer(L, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        return g
+
     def capture(layer_list, with_events=False):
         graphs, evs = [], []
         for L in layer_list:
@@ -311,41 +321,44 @@ def run_spense(args):
         torch.cuda.synchronize()
         return graphs, evs
 
-    def timed(graphs, steps, warmup, clocks=None):
-        for i in range(warmup):
-            graphs[i % len(graphs)].replay()
+    def timed(graphs, chain, steps, warmup, clocks=None):
+        # Steps run as whole-stack graphs (all rotated layers back to back, so
+        # each launch overlaps the previous one's tail); a remainder of fewer
+        # than `layers` steps uses the per-layer graphs.
+        def run(n):
+            for _ in range(n // len(graphs)):
+                chain.replay()
+            for i in range(n % len(graphs)):
+                graphs[i].replay()
+        run(warmup)
         torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(ranks)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         w0 = time.time()
         e0.record()
-        for i in range(steps):
-            graphs[i % len(graphs)].replay()
+        run(steps)
         e1.record()
         torch.cuda.synchronize()
         if clocks is not None:
             clocks.mark(w0, time.time())
-        if world > 1:
-            dist.barrier()
+        replicas.barrier(ranks)
         return e0.elapsed_time(e1) / 1e3  # seconds
 
     g_sp, _ = capture(layers_sp)
     g_dn, _ = capture(layers_dn)
+    c_sp = capture_chain(layers_sp)
+    c_dn = capture_chain(layers_dn)
 
     with ClockSampler(local) as clocks:
-        t_sp = timed(g_sp, args.steps, args.warmup, clocks)
-    t_dn = timed(g_dn, args.steps, args.warmup)
+        t_sp = timed(g_sp, c_sp, args.steps, args.warmup, clocks)
+    t_dn = timed(g_dn, c_dn, args.steps, args.warmup)
 
-    if world > 1:
-        t = torch.tensor([t_sp, t_dn], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_sp, t_dn = t.tolist()
+    t_sp, t_dn = replicas.max_over_ranks(ranks, [t_sp, t_dn], device=dev)
 
     per_step = step_bytes(args)
-    value = per_step * args.steps * world / t_sp / 1e9
+    value = replicas.job_rate(per_step * args.steps, world, t_sp) / 1e9
     launches = args.steps * len(GROUPS)
 
     # ---- dominant kernel: per-launch device time from events captured around each launch
@@ -385,8 +398,7 @@ def run_spense(args):
     e2e_steps = max(4, min(args.steps, 200))
     for i in range(min(args.warmup, 8)):
         e2e_step(layers_sp[i % args.layers])
-    if world > 1:
-        dist.barrier()
+    replicas.barrier(ranks)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -394,14 +406,10 @@ def run_spense(args):
         e2e_step(layers_sp[i % args.layers])
     e1.record()
     torch.cuda.synchronize()
-    t_e2e = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_e2e = t.item()
+    t_e2e = replicas.max_over_ranks(ranks, [e0.elapsed_time(e1) / 1e3], device=dev)[0]
     h2d = sum(M * SHAPES[g[0]][2] + 4 * M for g in GROUPS)
     d2h = sum(2 * M * n for _, n, _ in SHAPES)
-    e2e_value = per_step * e2e_steps * world / t_e2e / 1e9
+    e2e_value = replicas.job_rate(per_step * e2e_steps, world, t_e2e) / 1e9
 
     status = spense.workspace_status(ws)
     if status != 0:
@@ -441,10 +449,8 @@ def run_spense(args):
     for L in layers_sp + layers_dn:
         for p in L:
             p.free()
-    if world > 1:
-        dist.barrier()
-        del g_sp, g_dn
-        dist.destroy_process_group()
+    del g_sp, g_dn, c_sp, c_dn  # graphs are released before the process group goes away
+    replicas.finalize(ranks)
     return 0
 
 

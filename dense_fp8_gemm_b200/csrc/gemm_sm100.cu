@@ -241,7 +241,20 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     // (the packed weights never depend on it), the activation tiles after.
     // With two producer warps (warps 0 and 6) each issues every other block:
     // the copy engine serves the two issue streams concurrently.
-    if (lane == 0) {
+    if (lane == 0 && p.test_gate != nullptr) {
+      // Test of the failure path: wait (bounded) on a word nothing sets, before
+      // any copy is issued, so the timeout leaves no transfer in flight.
+      const uint64_t t0 = ptx::globaltimer();
+      while (*reinterpret_cast<const volatile unsigned int*>(p.test_gate) == 0u) {
+        if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+          atomicOr(p.status, SPENSE_DEVICE_TIMEOUT_PRODUCER);
+          *abort_flag = 1;
+          break;
+        }
+        __nanosleep(1000);
+      }
+    }
+    if (lane == 0 && !*abort_flag) {
       const int np = p.producers;
       const int me = warp == 0 ? 0 : 1;
       const uint64_t pol_w = ptx::policy_evict_first();

@@ -356,6 +356,10 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
   p.bulk_split = pl.bulk_split;
   p.producers = pl.producers;
   p.cluster = pl.cluster;
+  // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
+  // the workspace, which nothing sets, so every launch ends by timeout.
+  static const bool stall = env_int("SPENSE_TEST_STALL", 0, 0, 1) == 1;
+  p.test_gate = stall ? reinterpret_cast<const unsigned int*>(ws + 64) : nullptr;
   cudaError_t e = launch_gemm(map, p, pl.smem_bytes, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return SPENSE_OK;
@@ -523,6 +527,7 @@ size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M) {
 spense_status spense_gemm_grouped(const spense_packed* const* Wps, int count, const uint8_t* X,
                                   const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
                                   size_t workspace_bytes, void* stream_v) {
+  if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
   if (X == nullptr || x_scale == nullptr || Ys == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
   if (!aligned(X, 16) || !aligned(x_scale, 4))
     return fail(SPENSE_ERR_ALIGN, "X must be 16-byte aligned, x_scale 4-byte aligned");

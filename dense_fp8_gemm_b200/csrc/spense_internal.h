@@ -87,6 +87,7 @@ struct GemmParams {
   int bulk_split;  // weight block copied as this many bulk copies (1, 2 or 4)
   int producers;   // loader warps (1 or 2)
   int cluster;     // > 1: CTAs of a cluster split one tile's K and reduce through shared memory
+  const unsigned int* test_gate;  // test only: loaders wait (bounded) until this word is nonzero
 };
 
 // Kernels (defined in the .cu files).

@@ -279,3 +279,19 @@ def test_grouped_rejects_mismatched_layouts():
     with pytest.raises(spense.SpenseError) as ei:
         spense.gemm_grouped([a, b], _dev(X), _dev(s_x), workspace=spense.new_workspace(1 << 20))
     assert ei.value.code == 1
+
+
+def test_gemm_rejects_small_workspace_and_bad_token_count():
+    M, N, K, Kd = 4, 256, 512, 128
+    X, s_x, W, s_w, _ = _make(88, M, N, K, Kd)
+    pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd)
+    need = spense.workspace_size(pw, M)
+    small = spense.new_workspace(need - 256)
+    with pytest.raises(spense.SpenseError) as ei:
+        spense.gemm(pw, _dev(X), _dev(s_x), workspace=small)
+    assert ei.value.code == 7
+    empty = torch.empty((0, K), dtype=torch.uint8, device="cuda")
+    with pytest.raises(spense.SpenseError) as ei:
+        spense.gemm(pw, empty, _dev(s_x[:0]), Y=torch.empty((1, N), dtype=torch.bfloat16, device="cuda"),
+                    workspace=spense.new_workspace(need))
+    assert ei.value.code == 2
