@@ -57,7 +57,9 @@ struct alignas(8) Barriers {
   uint32_t tmem_base;
   int abort_flag;
   int fix_flag;
+  float sx[kMaxTokenTile];  // per-token scales of the token tile being finished
 };
+static_assert(sizeof(Barriers) <= kBarrierBytes, "barrier area too small");
 
 __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, unsigned int* status,
                                          unsigned int code, volatile int* abort_flag) {
@@ -192,7 +194,9 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  Barriers* bars = reinterpret_cast<Barriers*>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
+  // [stage ring][cluster receive area][barriers]
+  const uint32_t recv_off = static_cast<uint32_t>(p.stages) * p.stage_bytes;
+  Barriers* bars = reinterpret_cast<Barriers*>(smem + recv_off + p.recv_bytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
       ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), 128);
     }
-    ptx::mbar_init(ptx::smem_addr(&bars->peer_done), p.cluster > 1 ? p.cluster - 1 : 1);
+    ptx::mbar_init(ptx::smem_addr(&bars->peer_done), p.cluster > 1 ? 128 * (p.cluster - 1) : 1);
     bars->abort_flag = 0;
     bars->fix_flag = 0;
     ptx::fence_mbar_init();
@@ -376,6 +380,16 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
+    // Token scales of the current token tile, staged in shared memory before
+    // the accumulator is ready so no global load sits on the epilogue's path.
+    int staged_m0 = -1;
+    auto stage_sx = [&](int m0) {
+      if (m0 == staged_m0) return;
+      ptx::named_bar_sync(1, 128);  // earlier readers are done
+      for (int i = et; i < p.npad; i += 128) bars->sx[i] = (m0 + i < p.M) ? __ldg(p.s_x + m0 + i) : 0.0f;
+      ptx::named_bar_sync(1, 128);
+      staged_m0 = m0;
+    };
 
     // Sum the contributors' partials of tile t in CTA order and store Y. Every
     // contributor after g_lo starts inside tile t, so its partial is in slot
@@ -383,6 +397,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     auto finish_tile = [&](int t) {
       const int n_tile = t / p.m_tiles;
       const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      stage_sx(m0);
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
       const int n = (n_tile - mb.tile_begin) * kTileRows + row;
@@ -437,7 +452,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             for (int i = 0; i < 4; ++i) {
               const int m = c0 + 4 * q + i;
               if (q < nq && m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(r4[i] * sw * __ldg(p.s_x + m0 + m));
+                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] =
+                    to_bf16_bits(r4[i] * sw * (m0 == staged_m0 ? bars->sx[m] : __ldg(p.s_x + m0 + m)));
             }
           }
         }
@@ -452,38 +468,44 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     int npending = 0;
     if (p.cluster > 1 && units.count == 1) {
       // Cluster split: the S CTAs of a cluster hold consecutive K ranges of one
-      // tile. Peers leave their fp32 partial in their own (now idle) stage
-      // memory and signal rank 0, which adds them in rank order through
-      // distributed shared memory and stores Y.
+      // tile. Peers push their fp32 partial into rank 0's receive area over
+      // distributed shared memory and exit; rank 0 adds them in rank order
+      // and stores Y.
       int t, j0, j1;
       units.get(0, t, j0, j1);
+      const int n_tile = t / p.m_tiles;
+      const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      const GemmMember& mb = p.mem[member_of(p, n_tile)];
+      const int m_valid = min(p.npad, p.M - m0);
+      const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+      const bool row_ok = n < mb.N;
+      const uint32_t rank = ptx::cluster_ctarank();
+      const float sw = (row_ok && rank == 0) ? __ldg(mb.s_w + n) : 0.0f;
+      if (rank == 0) stage_sx(m0);
       const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[0]), 0, p.status,
                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
       if (__all_sync(0xffffffffu, got)) {
         ptx::tc_fence_after();
-        const int n_tile = t / p.m_tiles;
-        const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
-        const GemmMember& mb = p.mem[member_of(p, n_tile)];
-        const int m_valid = min(p.npad, p.M - m0);
-        const int n = (n_tile - mb.tile_begin) * kTileRows + row;
-        const bool row_ok = n < mb.N;
-        const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
-        const uint32_t rank = ptx::cluster_ctarank();
-        const uint32_t part_s = smem_base + static_cast<uint32_t>(row * p.npad) * 4u;
+        // Receive slot of peer r in rank 0: [r - 1][row][npad] floats.
+        const uint32_t slot_bytes = static_cast<uint32_t>(kTileRows * p.npad) * 4u;
+        const uint32_t row_off = static_cast<uint32_t>(row * p.npad) * 4u;
         if (rank != 0) {
+          // Push this CTA's partial into rank 0's receive area, then signal
+          // (each thread releases its own stores at cluster scope).
+          const uint32_t dst0 =
+              ptx::mapa(smem_base + recv_off + (rank - 1) * slot_bytes + row_off, 0);
           for (int c0 = 0; c0 < m_valid; c0 += 16) {
             uint32_t v[16];
             ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c0), v);
             ptx::tmem_ld_wait();
 #pragma unroll
             for (int q = 0; q < 4; ++q)
-              ptx::st_smem_v4(part_s + static_cast<uint32_t>(c0 + 4 * q) * 4u,
-                              make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+              ptx::st_dsmem_v4(dst0 + static_cast<uint32_t>(c0 + 4 * q) * 4u,
+                               make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                           __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
           }
           ptx::tc_fence_before();
-          ptx::named_bar_sync(1, 128);
-          if (et == 0) ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_addr(&bars->peer_done), 0));
+          ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_addr(&bars->peer_done), 0));
         } else if (wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status, SPENSE_DEVICE_TIMEOUT_EPILOGUE,
                                     abort_flag)) {
           for (int c0 = 0; c0 < m_valid; c0 += 16) {
@@ -494,16 +516,14 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
 #pragma unroll
             for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
             for (int r = 1; r < p.cluster; ++r) {
-              const uint32_t src = ptx::mapa(part_s + static_cast<uint32_t>(c0) * 4u, static_cast<uint32_t>(r));
-              float4 b[4];
-#pragma unroll
-              for (int q = 0; q < 4; ++q) b[q] = ptx::ld_dsmem_v4(src + 16u * q);
+              const uint32_t src = smem_base + recv_off + (r - 1) * slot_bytes + row_off + static_cast<uint32_t>(c0) * 4u;
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                a[4 * q] += b[q].x;
-                a[4 * q + 1] += b[q].y;
-                a[4 * q + 2] += b[q].z;
-                a[4 * q + 3] += b[q].w;
+                const float4 b = ptx::ld_smem_v4(src + 16u * q);
+                a[4 * q] += b.x;
+                a[4 * q + 1] += b.y;
+                a[4 * q + 2] += b.z;
+                a[4 * q + 3] += b.w;
               }
             }
             if (row_ok) {
@@ -511,7 +531,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
               for (int i = 0; i < 16; ++i) {
                 const int m = c0 + i;
                 if (m < m_valid)
-                  mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(a[i] * sw * __ldg(p.s_x + m0 + m));
+                  mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(a[i] * sw * bars->sx[m]);
               }
             }
           }
@@ -524,18 +544,19 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       units.get(u, t, j0, j1);
       const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
       const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
-      const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
-                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
-      ptx::tc_fence_after();
       const int n_tile = t / p.m_tiles;
       const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
       const int n = (n_tile - mb.tile_begin) * kTileRows + row;
       const bool row_ok = n < mb.N;
-      const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
       const bool whole = (j0 == 0 && j1 == nblk);
+      const float sw = (row_ok && whole) ? __ldg(mb.s_w + n) : 0.0f;
+      if (whole) stage_sx(m0);
+      const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
+                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
+      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
+      ptx::tc_fence_after();
       const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
       // Partials are stored [CTA][slot][row][npad]: slot 0 for the tile holding the
       // CTA's first block, slot 1 for the tile holding its last block.
@@ -554,8 +575,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             for (int i = 0; i < 16; ++i) {
               const int m = c0 + i;
               if (m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] =
-                    to_bf16_bits(__uint_as_float(v[i]) * sw * __ldg(p.s_x + m0 + m));
+                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(__uint_as_float(v[i]) * sw * bars->sx[m]);
             }
           }
         } else {
@@ -600,7 +620,15 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
-  if (p.cluster > 1) ptx::cluster_sync();  // peers keep their shared memory until rank 0 has read it
+  if (p.cluster > 1) {
+    // Peers leave as soon as their partial is pushed; rank 0 waits until every
+    // peer that has not exited has arrived, so it never exits while a peer
+    // may still write into its shared memory.
+    if (ptx::cluster_ctarank() == 0)
+      ptx::cluster_sync();
+    else
+      ptx::cluster_arrive();
+  }
   if (warp == 1) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem_base, p.tmem_cols);

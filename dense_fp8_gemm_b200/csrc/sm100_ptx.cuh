@@ -227,10 +227,29 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
   return v;
 }
 
+// Store to another CTA's shared memory (address from mapa).
+__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y),
+               "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ float4 ld_smem_v4(uint32_t saddr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(saddr)
+               : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void st_smem_v4(uint32_t saddr, float4 v) {
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "f"(v.x), "f"(v.y), "f"(v.z),
                "f"(v.w)
                : "memory");
+}
+
+// Arrive on the cluster barrier without waiting (releases prior writes).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 
 // Whole-cluster barrier (every thread of every CTA of the cluster).

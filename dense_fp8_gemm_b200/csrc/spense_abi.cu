@@ -196,7 +196,7 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   pl.producers = producers();
   pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.nsb > 0 ? 256u : 128u);
   pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.nsb > 0 ? kMetaBlockBytes : 0);
-  const uint32_t reserve = 1024 + 512;  // alignment slack + barriers
+  const uint32_t reserve = 1024 + kBarrierBytes;  // alignment slack + barrier area
   for (int cps = ctas_per_sm(); cps >= 1; --cps) {
     const uint32_t smem_budget = gemm_max_smem() / cps - (cps > 1 ? 1024u : 0u);
     const uint32_t tmem_budget = 512u / cps;
@@ -238,6 +238,20 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
       }
     }
   }
+  pl.recv_bytes = 0;
+  if (pl.cluster > 1) {
+    // Rank 0 receives S - 1 partials of 128 rows x npad floats; the ring gives
+    // up stages for it (at least two must remain).
+    pl.recv_bytes = static_cast<uint32_t>(pl.cluster - 1) * kTileRows * pl.npad * 4u;
+    const uint32_t smem_budget = gemm_max_smem() / pl.ctas_per_sm - (pl.ctas_per_sm > 1 ? 1024u : 0u);
+    if (smem_budget < reserve + pl.recv_bytes + 2 * pl.stage_bytes) {
+      pl.cluster = 1;
+      pl.recv_bytes = 0;
+    } else {
+      pl.stages = static_cast<int>(
+          std::min<uint32_t>(kMaxStages, (smem_budget - reserve - pl.recv_bytes) / pl.stage_bytes));
+    }
+  }
   if (pl.cluster > 1) {
     pl.grid = pl.tiles * pl.cluster;
     for (int g = 0; g <= pl.grid; ++g) {
@@ -254,7 +268,7 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
       pl.cta_start[g] = static_cast<int>(t * nblk + block_at(c - t * pl.tile_cost));
     }
   }
-  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
+  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes + pl.recv_bytes;
   int64_t n_sum = 0;
   for (int i = 0; i < count; ++i) n_sum += hs[i]->N;
   WorkspaceLayout& w = pl.ws;
@@ -356,6 +370,7 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
   p.bulk_split = pl.bulk_split;
   p.producers = pl.producers;
   p.cluster = pl.cluster;
+  p.recv_bytes = pl.recv_bytes;
   // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
   // the workspace, which nothing sets, so every launch ends by timeout.
   static const bool stall = env_int("SPENSE_TEST_STALL", 0, 0, 1) == 1;

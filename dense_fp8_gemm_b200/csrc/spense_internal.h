@@ -21,6 +21,7 @@ constexpr int kCostDense = 4;           // ... of a dense block (16 KiB)
 constexpr int kGemmThreads = 192;       // warp 0 loads, warp 1 issues MMAs, warps 2-5 epilogue
 constexpr int kGemmThreadsMax = 224;    // plus warp 6 as a second loader
 constexpr int kMaxStages = 12;
+constexpr uint32_t kBarrierBytes = 2048;  // mbarriers, flags and staged token scales
 
 // Workspace layout: [header 256 B][counters][partials][gathered X][host staging]
 struct WorkspaceLayout {
@@ -55,6 +56,7 @@ struct GemmPlan {
   int bulk_split;
   int producers;
   int cluster;
+  uint32_t recv_bytes;
   int cta_start[kMaxGrid + 1];  // first linear block of each CTA; [grid] = total blocks
   WorkspaceLayout ws;
 };
@@ -88,6 +90,7 @@ struct GemmParams {
   int producers;   // loader warps (1 or 2)
   int cluster;     // > 1: CTAs of a cluster split one tile's K and reduce through shared memory
   const unsigned int* test_gate;  // test only: loaders wait (bounded) until this word is nonzero
+  uint32_t recv_bytes;            // cluster mode: rank 0's receive area for the peers' partials
 };
 
 // Kernels (defined in the .cu files).
