@@ -15,10 +15,11 @@
 // one activation tensor (for example q, k and v projections); their row tiles
 // are laid end to end.
 //
-// Roles (one CTA per SM, 192 threads):
-//   warp 0   producer: bulk copies of the packed weight blocks (values,
+// Roles (up to two CTAs per SM, 192 or 224 threads):
+//   warps 0, 6 producers: bulk copies of the packed weight blocks (values,
 //            metadata, dense columns) and 2-D TMA loads of the activation tile
-//            into a ring of shared-memory stages;
+//            into a ring of shared-memory stages; with two producer warps
+//            each issues every other block;
 //   warp 1   allocates tensor memory; one lane copies the metadata into tensor
 //            memory (tcgen05.cp) and issues the MMAs;
 //   warps 2-5 epilogue: tensor memory -> registers, scales, bf16 stores, or
@@ -32,6 +33,11 @@
 // whole tiles instead of forming the kernel's tail. A shared tile is finished
 // by the last contributor to arrive, which sums every contributor's partial in
 // CTA order, so the result does not depend on arrival order.
+//
+// Launches with few tiles use a cluster split instead: the S CTAs of a cluster
+// (S = 2, 4 or 8) stream consecutive K ranges of one tile; the peers send
+// their fp32 partials into rank 0's shared memory with asynchronous
+// distributed-shared-memory stores, and rank 0 adds them in rank order.
 //
 // Every wait is bounded (1.5 s by %globaltimer); on expiry the kernel records a
 // code in the workspace status word and all roles leave their loops.
@@ -53,7 +59,7 @@ struct alignas(8) Barriers {
   uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
-  uint64_t peer_done;  // cluster mode: one arrival per peer CTA whose partial is ready
+  uint64_t peer_done;  // cluster mode, rank 0: completes when every peer's partial has landed
   uint32_t tmem_base;
   int abort_flag;
   int fix_flag;
@@ -211,7 +217,16 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
       ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), 128);
     }
-    ptx::mbar_init(ptx::smem_addr(&bars->peer_done), p.cluster > 1 ? 128 * (p.cluster - 1) : 1);
+    ptx::mbar_init(ptx::smem_addr(&bars->peer_done), 1);
+    if (p.cluster > 1 && ptx::cluster_ctarank() == 0) {
+      // Rank 0 expects every peer's partial of its tile (whole 16-token
+      // chunks up to the valid tokens) as asynchronous stores; this is done
+      // before the cluster barrier below, so before any peer can send.
+      const int t = p.cta_start[blockIdx.x] / (p.nsb + p.ndb);
+      const int m_valid = min(p.npad, p.M - (t % p.m_tiles) * kMaxTokenTile);
+      const uint32_t bytes = static_cast<uint32_t>((p.cluster - 1) * ((m_valid + 15) >> 4)) * kTileRows * 64u;
+      ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->peer_done), bytes);
+    }
     bars->abort_flag = 0;
     bars->fix_flag = 0;
     ptx::fence_mbar_init();
@@ -468,47 +483,60 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     int npending = 0;
     if (p.cluster > 1 && units.count == 1) {
       // Cluster split: the S CTAs of a cluster hold consecutive K ranges of one
-      // tile. Peers push their fp32 partial into rank 0's receive area over
-      // distributed shared memory and exit; rank 0 adds them in rank order
-      // and stores Y.
+      // tile. Peers push their fp32 partial into rank 0's receive area with
+      // asynchronous stores that count down rank 0's peer_done barrier, and
+      // exit; rank 0 adds them in rank order and stores Y.
       int t, j0, j1;
       units.get(0, t, j0, j1);
       const int n_tile = t / p.m_tiles;
       const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
-      const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+      const int nchunk = (m_valid + 15) >> 4;
+      const int n_base = (n_tile - mb.tile_begin) * kTileRows;
+      const int n = n_base + row;
       const bool row_ok = n < mb.N;
       const uint32_t rank = ptx::cluster_ctarank();
       const float sw = (row_ok && rank == 0) ? __ldg(mb.s_w + n) : 0.0f;
       if (rank == 0) stage_sx(m0);
       const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[0]), 0, p.status,
                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
-      if (__all_sync(0xffffffffu, got)) {
+      // Rank 0 also needs every peer's partial; its 128 threads take one
+      // decision (they meet at named barriers below).
+      const bool ready =
+          rank != 0 ? __all_sync(0xffffffffu, got)
+                    : ptx::named_bar_and(1, 128,
+                                         got && wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status,
+                                                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag));
+      if (ready) {
         ptx::tc_fence_after();
-        // Receive slot of peer r in rank 0: [r - 1][row][npad] floats.
+        // Receive slot of peer r in rank 0: [r - 1][chunk][row][16 floats]; the
+        // four 16-byte pieces of a row are rotated by (row >> 1) & 3 so that
+        // eight consecutive rows cover all shared-memory banks.
         const uint32_t slot_bytes = static_cast<uint32_t>(kTileRows * p.npad) * 4u;
-        const uint32_t row_off = static_cast<uint32_t>(row * p.npad) * 4u;
+        const uint32_t row_off = static_cast<uint32_t>(row) * 64u;
+        const uint32_t rot = static_cast<uint32_t>(row >> 1) & 3u;
         if (rank != 0) {
-          // Push this CTA's partial into rank 0's receive area, then signal
-          // (each thread releases its own stores at cluster scope).
-          const uint32_t dst0 =
-              ptx::mapa(smem_base + recv_off + (rank - 1) * slot_bytes + row_off, 0);
-          for (int c0 = 0; c0 < m_valid; c0 += 16) {
+          const uint32_t dst0 = ptx::mapa(smem_base + recv_off + (rank - 1) * slot_bytes + row_off, 0);
+          const uint32_t bar0 = ptx::mapa(ptx::smem_addr(&bars->peer_done), 0);
+          for (int c = 0; c < nchunk; ++c) {
             uint32_t v[16];
-            ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c0), v);
+            ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c * 16), v);
             ptx::tmem_ld_wait();
+            const uint32_t dst = dst0 + static_cast<uint32_t>(c) * (kTileRows * 64u);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              ptx::st_dsmem_v4(dst0 + static_cast<uint32_t>(c0 + 4 * q) * 4u,
-                               make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                           __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+            for (uint32_t q = 0; q < 4; ++q)
+              ptx::st_async_v4(dst + ((q ^ rot) << 4), v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], bar0);
           }
           ptx::tc_fence_before();
-          ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_addr(&bars->peer_done), 0));
-        } else if (wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status, SPENSE_DEVICE_TIMEOUT_EPILOGUE,
-                                    abort_flag)) {
-          for (int c0 = 0; c0 < m_valid; c0 += 16) {
+        } else {
+          // Y tile staged as [16 tokens][128 rows] bf16 in the first ring stage
+          // (idle: every copy has landed and every MMA has completed), then
+          // written with 16-byte stores when the tile's rows are all in range.
+          const bool vec = (n_base + kTileRows <= mb.N) && (mb.N % 8 == 0);
+          uint16_t* ystage = reinterpret_cast<uint16_t*>(smem);
+          for (int c = 0; c < nchunk; ++c) {
+            const int c0 = c * 16;
             uint32_t v[16];
             ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c0), v);
             ptx::tmem_ld_wait();
@@ -516,17 +544,31 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
 #pragma unroll
             for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
             for (int r = 1; r < p.cluster; ++r) {
-              const uint32_t src = smem_base + recv_off + (r - 1) * slot_bytes + row_off + static_cast<uint32_t>(c0) * 4u;
+              const uint32_t src = smem_base + recv_off + (r - 1) * slot_bytes +
+                                   static_cast<uint32_t>(c) * (kTileRows * 64u) + row_off;
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float4 b = ptx::ld_smem_v4(src + 16u * q);
+              for (uint32_t q = 0; q < 4; ++q) {
+                const float4 b = ptx::ld_smem_v4(src + ((q ^ rot) << 4));
                 a[4 * q] += b.x;
                 a[4 * q + 1] += b.y;
                 a[4 * q + 2] += b.z;
                 a[4 * q + 3] += b.w;
               }
             }
-            if (row_ok) {
+            if (vec) {
+              if (c > 0) ptx::named_bar_sync(1, 128);  // the previous chunk's readers are done
+#pragma unroll
+              for (int i = 0; i < 16; ++i) ystage[i * kTileRows + row] = to_bf16_bits(a[i] * sw * bars->sx[c0 + i]);
+              ptx::named_bar_sync(1, 128);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int idx = et + 128 * h;  // 16-byte piece: token idx / 16, rows 8 * (idx % 16) ..
+                const int m = c0 + (idx >> 4);
+                if (m < m_valid)
+                  ptx::st_global_v4(mb.y + static_cast<size_t>(m0 + m) * mb.N + n_base + 8 * (idx & 15),
+                                    reinterpret_cast<const uint4*>(ystage)[idx]);
+              }
+            } else if (row_ok) {
 #pragma unroll
               for (int i = 0; i < 16; ++i) {
                 const int m = c0 + i;
@@ -555,7 +597,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       if (whole) stage_sx(m0);
       const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
-      if (!__all_sync(0xffffffffu, got)) break;  // warp-uniform: tcgen05.ld needs the whole warp
+      // One decision for the 128 threads: they meet at named barriers below.
+      if (!ptx::named_bar_and(1, 128, got)) break;
       ptx::tc_fence_after();
       const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
       // Partials are stored [CTA][slot][row][npad]: slot 0 for the tile holding the
@@ -621,13 +664,19 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   ptx::tc_fence_before();
   __syncthreads();
   if (p.cluster > 1) {
-    // Peers leave as soon as their partial is pushed; rank 0 waits until every
-    // peer that has not exited has arrived, so it never exits while a peer
-    // may still write into its shared memory.
-    if (ptx::cluster_ctarank() == 0)
-      ptx::cluster_sync();
-    else
+    // Rank 0 normally exits once every peer's partial has landed (nothing
+    // else touches its shared memory). After a failed wait it first gives
+    // the peers' stores time to land (bounded) and waits for every peer to
+    // reach this point, so it never exits while a peer may still write to it.
+    if (ptx::cluster_ctarank() != 0) {
       ptx::cluster_arrive();
+    } else if (*abort_flag) {
+      const uint64_t t0 = ptx::globaltimer();
+      while (!ptx::mbar_try_wait_cluster(ptx::smem_addr(&bars->peer_done), 0) &&
+             ptx::globaltimer() - t0 < kWaitLimitNs) {
+      }
+      ptx::cluster_sync();
+    }
   }
   if (warp == 1) {
     ptx::tc_fence_after();
