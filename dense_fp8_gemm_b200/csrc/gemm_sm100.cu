@@ -207,8 +207,27 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = blockIdx.x;
+  // Let the next kernel in the stream start launching: its CTAs take SMs as
+  // this grid's CTAs exit and wait (griddepcontrol.wait) before reading
+  // anything this grid writes.
+  ptx::griddep_launch_dependents();
+  const int nblk = p.nsb + p.ndb;
+  const int b0 = p.cta_start[g];
+  const int b1 = p.cta_start[g + 1];
 
+  if (warp >= 2 && warp <= 5) {
+    // The epilogue warps are idle during set-up: they touch the whole
+    // parameter block once, so the constant-cache misses are taken in one
+    // parallel round trip instead of one after another on the producers'
+    // path to their first copy.
+    const uint32_t* pw = reinterpret_cast<const uint32_t*>(&p);
+    uint32_t acc = 0;
+    for (uint32_t i = static_cast<uint32_t>(threadIdx.x - 64) * 8u; i < sizeof(GemmParams) / 4; i += 1024u)
+      acc ^= pw[i];
+    asm volatile("" ::"r"(acc));
+  }
   if (threadIdx.x == 0) {
+    ptx::prefetch_tensormap(&tmap_x);
     for (int s = 0; s < p.stages; ++s) {
       ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
       ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
@@ -220,9 +239,10 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     ptx::mbar_init(ptx::smem_addr(&bars->peer_done), 1);
     if (p.cluster > 1 && ptx::cluster_ctarank() == 0) {
       // Rank 0 expects every peer's partial of its tile (whole 16-token
-      // chunks up to the valid tokens) as asynchronous stores; this is done
-      // before the cluster barrier below, so before any peer can send.
-      const int t = p.cta_start[blockIdx.x] / (p.nsb + p.ndb);
+      // chunks up to the valid tokens) as asynchronous stores. This precedes
+      // its arrival on the cluster barrier, which every peer waits for
+      // before its first store.
+      const int t = b0 / nblk;
       const int m_valid = min(p.npad, p.M - (t % p.m_tiles) * kMaxTokenTile);
       const uint32_t bytes = static_cast<uint32_t>((p.cluster - 1) * ((m_valid + 15) >> 4)) * kTileRows * 64u;
       ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->peer_done), bytes);
@@ -231,27 +251,27 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     bars->fix_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) ptx::prefetch_tensormap(&tmap_x);
   if (warp == 1) {
     ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), p.tmem_cols);
     ptx::tmem_relinquish();
   }
-  ptx::tc_fence_before();
-  __syncthreads();
-  if (p.cluster > 1) ptx::cluster_sync();  // peers' barriers are initialised before any remote arrive
-  ptx::tc_fence_after();
-  const uint32_t tmem_base = bars->tmem_base;
+  // Set-up barriers: the producers only need the mbarriers, so warp 0 (which
+  // initialised them) releases the second producer warp (named barrier 2)
+  // and the MMA and epilogue warps (named barrier 3, which also publishes the
+  // tensor-memory address) without waiting for them. Every thread arrives on
+  // the cluster barrier once here; a peer waits on it before its first store
+  // into rank 0.
+  auto setup_wait = [&]() -> uint32_t {
+    if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+    ptx::tc_fence_before();
+    ptx::named_bar_sync(3, kGemmThreads);
+    ptx::tc_fence_after();
+    return bars->tmem_base;
+  };
   volatile int* abort_flag = &bars->abort_flag;
-  // Let the next kernel in the stream start launching: its CTAs take SMs as
-  // this grid's CTAs exit and wait (griddepcontrol.wait) before reading
-  // anything this grid writes.
-  ptx::griddep_launch_dependents();
-
-  const int nblk = p.nsb + p.ndb;
-  const int b0 = p.cta_start[g];
-  const int b1 = p.cta_start[g + 1];
   const Units units(b0, b1, nblk);
   const uint32_t smem_base = ptx::smem_addr(smem);
+  bool cluster_waited = false;  // this thread has waited on its set-up arrival
 
   if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------ producer(s)
@@ -260,6 +280,15 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     // (the packed weights never depend on it), the activation tiles after.
     // With two producer warps (warps 0 and 6) each issues every other block:
     // the copy engine serves the two issue streams concurrently.
+    if (warp == 0) {
+      __syncwarp();  // lane 0 initialised the barriers
+      if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+      ptx::named_bar_arrive(3, kGemmThreads);
+      if (p.producers > 1) ptx::named_bar_arrive(2, 64);
+    } else {
+      ptx::named_bar_sync(2, 64);
+      if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+    }
     if (lane == 0 && p.test_gate != nullptr) {
       // Test of the failure path: wait (bounded) on a word nothing sets, before
       // any copy is issued, so the timeout leaves no transfer in flight.
@@ -332,6 +361,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
+    const uint32_t tmem_base = setup_wait();
     if (lane == 0) {
       const uint32_t idesc_sp = ptx::idesc_f8(static_cast<uint32_t>(p.npad), true);
       const uint32_t idesc_d = ptx::idesc_f8(static_cast<uint32_t>(p.npad), false);
@@ -389,6 +419,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const uint32_t tmem_base = setup_wait();
     ptx::griddep_wait();  // s_x, Y and the workspace may belong to the previous grid
     const int et = threadIdx.x - 64;  // 0..127
     const int quarter = warp & 3;     // tensor-memory lane quarter this warp may read
@@ -517,6 +548,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         const uint32_t row_off = static_cast<uint32_t>(row) * 64u;
         const uint32_t rot = static_cast<uint32_t>(row >> 1) & 3u;
         if (rank != 0) {
+          ptx::cluster_wait();  // rank 0's barrier is initialised and expects the bytes
+          cluster_waited = true;
           const uint32_t dst0 = ptx::mapa(smem_base + recv_off + (rank - 1) * slot_bytes + row_off, 0);
           const uint32_t bar0 = ptx::mapa(ptx::smem_addr(&bars->peer_done), 0);
           for (int c = 0; c < nchunk; ++c) {
@@ -663,24 +696,29 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   __syncwarp();
   ptx::tc_fence_before();
   __syncthreads();
+  // Tensor memory is released before any cluster-barrier operation: a
+  // dealloc issued after an arrival was measured to stall for microseconds,
+  // keeping the CTA (and its SM slot) alive.
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(bars->tmem_base, p.tmem_cols);
+  }
   if (p.cluster > 1) {
     // Rank 0 normally exits once every peer's partial has landed (nothing
     // else touches its shared memory). After a failed wait it first gives
     // the peers' stores time to land (bounded) and waits for every peer to
     // reach this point, so it never exits while a peer may still write to it.
     if (ptx::cluster_ctarank() != 0) {
-      ptx::cluster_arrive();
+      if (!cluster_waited) ptx::cluster_wait();
+      ptx::cluster_arrive_relaxed();  // only rank 0's failure path waits for it
     } else if (*abort_flag) {
       const uint64_t t0 = ptx::globaltimer();
       while (!ptx::mbar_try_wait_cluster(ptx::smem_addr(&bars->peer_done), 0) &&
              ptx::globaltimer() - t0 < kWaitLimitNs) {
       }
+      ptx::cluster_wait();
       ptx::cluster_sync();
     }
-  }
-  if (warp == 1) {
-    ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 

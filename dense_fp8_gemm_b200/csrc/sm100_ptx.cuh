@@ -185,6 +185,12 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrive on a named barrier without waiting (the waiting side uses bar.sync
+// with the same thread count).
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Named barrier over n threads that also ANDs a predicate across them, so
 // the threads leave with the same decision.
 __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
@@ -281,6 +287,17 @@ __device__ __forceinline__ void st_smem_v4(uint32_t saddr, float4 v) {
 // Arrive on the cluster barrier without waiting (releases prior writes).
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+// Arrive on the cluster barrier without waiting and without ordering any
+// earlier memory access.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+
+// Wait for the cluster barrier phase this thread arrived on (acquire).
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Whole-cluster barrier (every thread of every CTA of the cluster).
