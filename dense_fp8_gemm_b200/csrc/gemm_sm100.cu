@@ -60,6 +60,7 @@ struct alignas(8) Barriers {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t peer_done;  // cluster mode, rank 0: completes when every peer's partial has landed
+  uint64_t ack;        // cluster mode, peers: rank 0 has received this CTA's partial
   uint32_t tmem_base;
   int abort_flag;
   int fix_flag;
@@ -237,9 +238,10 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), 128);
     }
     ptx::mbar_init(ptx::smem_addr(&bars->peer_done), 1);
+    ptx::mbar_init(ptx::smem_addr(&bars->ack), 1);
     if (p.cluster > 1 && ptx::cluster_ctarank() == 0) {
       // Rank 0 expects every peer's partial of its tile (whole 16-token
-      // chunks up to the valid tokens) as asynchronous stores. This precedes
+      // chunks up to the valid tokens) as one bulk copy per peer. This precedes
       // its arrival on the cluster barrier, which every peer waits for
       // before its first store.
       const int t = b0 / nblk;
@@ -271,7 +273,6 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   volatile int* abort_flag = &bars->abort_flag;
   const Units units(b0, b1, nblk);
   const uint32_t smem_base = ptx::smem_addr(smem);
-  bool cluster_waited = false;  // this thread has waited on its set-up arrival
 
   if (warp == 0 || warp == 6) {
     // ------------------------------------------------------------ producer(s)
@@ -344,6 +345,25 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       BlockWalker cw(units, p);
       for (int i = 0; i < pre; ++i, cw.advance(p))
         if (i % np == me) issue_w(cw, static_cast<uint32_t>(i));
+      if (p.l2_prefetch > 0) {
+        // The weights past the first ring's worth are pulled into L2 while
+        // this grid waits on the previous one, so the HBM keeps streaming
+        // through the previous grid's tail; the ring later reads them from L2.
+        BlockWalker cp = cw;
+        const int last = min(nb, pre + p.l2_prefetch);
+        for (int i = pre; i < last; ++i, cp.advance(p)) {
+          if (i % np != me) continue;
+          const GemmMember& mb = p.mem[cp.member];
+          if (cp.j < p.nsb) {
+            const size_t blk = static_cast<size_t>(cp.local_tile) * p.nsb + cp.j;
+            ptx::prefetch_l2_bulk(mb.vs_t + blk * kBlockBytes, kBlockBytes);
+            ptx::prefetch_l2_bulk(mb.e_t + blk * kMetaBlockBytes, kMetaBlockBytes);
+          } else {
+            const size_t blk = static_cast<size_t>(cp.local_tile) * p.ndb + (cp.j - p.nsb);
+            ptx::prefetch_l2_bulk(mb.wd_t + blk * kBlockBytes, kBlockBytes);
+          }
+        }
+      }
       ptx::griddep_wait();
       BlockWalker cx(units, p);
       for (int i = 0; i < pre; ++i, cx.advance(p))
@@ -514,9 +534,11 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     int npending = 0;
     if (p.cluster > 1 && units.count == 1) {
       // Cluster split: the S CTAs of a cluster hold consecutive K ranges of one
-      // tile. Peers push their fp32 partial into rank 0's receive area with
-      // asynchronous stores that count down rank 0's peer_done barrier, and
-      // exit; rank 0 adds them in rank order and stores Y.
+      // tile. Each peer stages its fp32 partial in its own (idle) ring and
+      // sends it to rank 0's receive area with one bulk copy that counts down
+      // rank 0's peer_done barrier. Rank 0 acknowledges on each peer's ack
+      // barrier (a peer's staging must outlive its copy), adds the partials
+      // in rank order and stores Y.
       int t, j0, j1;
       units.get(0, t, j0, j1);
       const int n_tile = t / p.m_tiles;
@@ -532,13 +554,12 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       if (rank == 0) stage_sx(m0);
       const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[0]), 0, p.status,
                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag);
-      // Rank 0 also needs every peer's partial; its 128 threads take one
+      // Rank 0 also needs every peer's partial. The 128 threads take one
       // decision (they meet at named barriers below).
-      const bool ready =
-          rank != 0 ? __all_sync(0xffffffffu, got)
-                    : ptx::named_bar_and(1, 128,
-                                         got && wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status,
-                                                                 SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag));
+      const bool ready = ptx::named_bar_and(
+          1, 128,
+          got && (rank != 0 || wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status,
+                                                SPENSE_DEVICE_TIMEOUT_EPILOGUE, abort_flag)));
       if (ready) {
         ptx::tc_fence_after();
         // Receive slot of peer r in rank 0: [r - 1][chunk][row][16 floats]; the
@@ -548,21 +569,37 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         const uint32_t row_off = static_cast<uint32_t>(row) * 64u;
         const uint32_t rot = static_cast<uint32_t>(row >> 1) & 3u;
         if (rank != 0) {
-          ptx::cluster_wait();  // rank 0's barrier is initialised and expects the bytes
-          cluster_waited = true;
-          const uint32_t dst0 = ptx::mapa(smem_base + recv_off + (rank - 1) * slot_bytes + row_off, 0);
-          const uint32_t bar0 = ptx::mapa(ptx::smem_addr(&bars->peer_done), 0);
+          // Rank 0's peer_done barrier is initialised and expects the bytes
+          // once every CTA of the cluster has arrived from its set-up.
+          ptx::cluster_wait();
+          // Staging: the receive layout, [chunk][row][16 floats] with rotated
+          // 16-byte pieces, from the start of this CTA's ring (every copy has
+          // landed and every MMA has completed).
           for (int c = 0; c < nchunk; ++c) {
             uint32_t v[16];
             ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c * 16), v);
             ptx::tmem_ld_wait();
-            const uint32_t dst = dst0 + static_cast<uint32_t>(c) * (kTileRows * 64u);
+            const uint32_t dst = smem_base + static_cast<uint32_t>(c) * (kTileRows * 64u) + row_off;
 #pragma unroll
             for (uint32_t q = 0; q < 4; ++q)
-              ptx::st_async_v4(dst + ((q ^ rot) << 4), v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3], bar0);
+              ptx::st_smem_v4(dst + ((q ^ rot) << 4),
+                              make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
           }
           ptx::tc_fence_before();
+          ptx::fence_proxy_async_smem();
+          ptx::named_bar_sync(1, 128);
+          if (et == 0) {
+            ptx::bulk_s2s_cluster(ptx::mapa(smem_base + recv_off + (rank - 1) * slot_bytes, 0), smem_base,
+                                  static_cast<uint32_t>(nchunk) * (kTileRows * 64u),
+                                  ptx::mapa(ptx::smem_addr(&bars->peer_done), 0));
+          }
         } else {
+          // Every copy has landed (so every peer is alive, waiting for this):
+          // release the peers.
+          if (et == 0)
+            for (int r = 1; r < p.cluster; ++r)
+              ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_addr(&bars->ack), static_cast<uint32_t>(r)));
           // Y tile staged as [16 tokens][128 rows] bf16 in the first ring stage
           // (idle: every copy has landed and every MMA has completed), then
           // written with 16-byte stores when the tile's rows are all in range.
@@ -704,20 +741,19 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     ptx::tmem_dealloc(bars->tmem_base, p.tmem_cols);
   }
   if (p.cluster > 1) {
-    // Rank 0 normally exits once every peer's partial has landed (nothing
-    // else touches its shared memory). After a failed wait it first gives
-    // the peers' stores time to land (bounded) and waits for every peer to
-    // reach this point, so it never exits while a peer may still write to it.
     if (ptx::cluster_ctarank() != 0) {
-      if (!cluster_waited) ptx::cluster_wait();
-      ptx::cluster_arrive_relaxed();  // only rank 0's failure path waits for it
+      // A peer's staged partial must outlive its bulk copy: wait (bounded)
+      // for rank 0's acknowledgement. Rank 0 only acknowledges on its success
+      // path; after a failure elsewhere the wait runs out and the peer leaves.
+      const uint64_t t0 = ptx::globaltimer();
+      while (!ptx::mbar_try_wait_cluster(ptx::smem_addr(&bars->ack), 0) && ptx::globaltimer() - t0 < kWaitLimitNs) {
+      }
     } else if (*abort_flag) {
+      // Rank 0 never exits while a peer's copy may still write into it.
       const uint64_t t0 = ptx::globaltimer();
       while (!ptx::mbar_try_wait_cluster(ptx::smem_addr(&bars->peer_done), 0) &&
              ptx::globaltimer() - t0 < kWaitLimitNs) {
       }
-      ptx::cluster_wait();
-      ptx::cluster_sync();
     }
   }
 }

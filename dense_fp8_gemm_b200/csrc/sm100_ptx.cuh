@@ -239,6 +239,30 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Bulk prefetch of global memory into L2 (no shared-memory destination);
+// address 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// Bulk copy from this CTA's shared memory into another CTA's shared memory
+// (dst and mbar from mapa); complete_tx(bytes) on that CTA's mbarrier when the
+// data has landed. The source must stay valid until then.
+__device__ __forceinline__ void bulk_s2s_cluster(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                 uint32_t mbar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst_cluster),
+      "r"(src), "r"(bytes), "r"(mbar_cluster)
+      : "memory");
+}
+
+// Orders this thread's generic-proxy shared-memory writes before later
+// async-proxy (bulk copy) reads of them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Asynchronous 16-byte store into another CTA's shared memory; on arrival it
 // performs complete_tx(16) on that CTA's mbarrier (both addresses from mapa).
 __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
@@ -298,6 +322,16 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 // Wait for the cluster barrier phase this thread arrived on (acquire).
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Per-thread form of cluster_wait (no warp convergence required).
+__device__ __forceinline__ void cluster_wait_thread() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Per-thread form of cluster_arrive_relaxed.
+__device__ __forceinline__ void cluster_arrive_thread_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
 }
 
 // Whole-cluster barrier (every thread of every CTA of the cluster).

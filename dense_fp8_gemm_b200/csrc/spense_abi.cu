@@ -137,6 +137,17 @@ int ctas_per_sm() {
   static const int v = env_int("SPENSE_CTAS_PER_SM", 2, 1, 2);
   return v;
 }
+// CTA slots per SM that one grid may fill (default: all of them); 1 leaves
+// room for the next grid in the stream to start beside this one.
+int grid_per_sm() {
+  static const int v = env_int("SPENSE_GRID_PER_SM", 2, 1, 2);
+  return v;
+}
+// Blocks per CTA prefetched into L2 at start (0 = none).
+int l2_prefetch_blocks() {
+  static const int v = env_int("SPENSE_L2_PREFETCH", 0, 0, 1 << 20);
+  return v;
+}
 int producers() {
   static const int v = env_int("SPENSE_PRODUCERS", 2, 1, 2);
   return v;
@@ -211,7 +222,8 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     pl.tmem_cols = cols;
     break;
   }
-  const long long slots = std::min<long long>(static_cast<long long>(sms) * pl.ctas_per_sm, kMaxGrid);
+  const long long slots =
+      std::min<long long>(static_cast<long long>(sms) * std::min(pl.ctas_per_sm, grid_per_sm()), kMaxGrid);
   // First block of a tile whose start weight is >= c (c within one tile).
   auto block_at = [&](long long c) {
     const long long sp = static_cast<long long>(kCostSparse) * pl.nsb;
@@ -371,6 +383,7 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
   p.producers = pl.producers;
   p.cluster = pl.cluster;
   p.recv_bytes = pl.recv_bytes;
+  p.l2_prefetch = l2_prefetch_blocks();
   // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
   // the workspace, which nothing sets, so every launch ends by timeout.
   static const bool stall = env_int("SPENSE_TEST_STALL", 0, 0, 1) == 1;

@@ -91,6 +91,7 @@ struct GemmParams {
   int cluster;     // > 1: CTAs of a cluster split one tile's K and reduce through shared memory
   const unsigned int* test_gate;  // test only: loaders wait (bounded) until this word is nonzero
   uint32_t recv_bytes;            // cluster mode: rank 0's receive area for the peers' partials
+  int l2_prefetch;                // blocks past the first ring's worth prefetched into L2 at start
 };
 
 // Kernels (defined in the .cu files).
