@@ -436,6 +436,14 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         if (!ok) break;
         ptx::mma_commit(ptx::smem_addr(&bars->acc_full[acc]));
       }
+      if (ok && p.cluster > 1 && ptx::cluster_ctarank() == 0 &&
+          wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status, SPENSE_DEVICE_TIMEOUT_EPILOGUE,
+                           abort_flag)) {
+        // Every peer's copy has landed (so every peer is alive, waiting for
+        // this): release them. Off the epilogue's path.
+        for (int r = 1; r < p.cluster; ++r)
+          ptx::mbar_arrive_remote_relaxed(ptx::mapa(ptx::smem_addr(&bars->ack), static_cast<uint32_t>(r)));
+      }
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -536,9 +544,9 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       // Cluster split: the S CTAs of a cluster hold consecutive K ranges of one
       // tile. Each peer stages its fp32 partial in its own (idle) ring and
       // sends it to rank 0's receive area with one bulk copy that counts down
-      // rank 0's peer_done barrier. Rank 0 acknowledges on each peer's ack
-      // barrier (a peer's staging must outlive its copy), adds the partials
-      // in rank order and stores Y.
+      // rank 0's peer_done barrier; rank 0 adds the partials in rank order
+      // and stores Y, while its MMA warp acknowledges the copies (a peer's
+      // staging must outlive its copy).
       int t, j0, j1;
       units.get(0, t, j0, j1);
       const int n_tile = t / p.m_tiles;
@@ -595,11 +603,6 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
                                   ptx::mapa(ptx::smem_addr(&bars->peer_done), 0));
           }
         } else {
-          // Every copy has landed (so every peer is alive, waiting for this):
-          // release the peers.
-          if (et == 0)
-            for (int r = 1; r < p.cluster; ++r)
-              ptx::mbar_arrive_remote(ptx::mapa(ptx::smem_addr(&bars->ack), static_cast<uint32_t>(r)));
           // Y tile staged as [16 tokens][128 rows] bf16 in the first ring stage
           // (idle: every copy has landed and every MMA has completed), then
           // written with 16-byte stores when the tile's rows are all in range.
