@@ -77,18 +77,27 @@ def step_bytes(args, dense=False):
     return total
 
 
+KERNEL_SOURCES = ("gemm_sm100.cu", "sm100_ptx.cuh", "spense_internal.h")
+
+
+def kernel_source_sha256():
+    """sha256 over the sources that define spense_gemm_kernel, in a fixed order."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "dense_fp8_gemm_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def read_traffic():
     """DRAM bytes per launch of spense_gemm_kernel from the committed ncu summary,
-    or None when the kernel source has changed since the counters were taken."""
-    import hashlib
+    or None when the kernel sources have changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "spense_gemm_attn32b_m16_traffic.txt")
-    src = os.path.join(ROOT, "dense_fp8_gemm_b200", "csrc", "gemm_sm100.cu")
     try:
         with open(path) as f:
             rec = json.load(f)
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        return rec["dram_bytes_per_launch_avg"] if rec["kernel_source_sha256"] == sha else None
+        return rec["dram_bytes_per_launch_avg"] if rec["kernel_source_sha256"] == kernel_source_sha256() else None
     except Exception:
         return None
 
