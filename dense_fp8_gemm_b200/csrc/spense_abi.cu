@@ -122,19 +122,26 @@ long long min_cta_weight() {
   return v;
 }
 
-// Tuning knobs read once from the environment: CTAs per SM (1 or 2, default 2),
-// loader warps per CTA (1 or 2, default 2) and how many bulk copies move one
-// 16 KiB weight block (1, 2 or 4, default 1). One SM's copy engine serves
-// several issue streams at once but one stream's copies one after another, so
-// two CTAs with two loader warps each keep four streams going per SM.
+// Tuning knobs read once from the environment: CTAs per SM (1, 2 or 0 =
+// automatic), loader warps per CTA (1 or 2, default 2) and how many bulk
+// copies move one 16 KiB weight block (1, 2 or 4, default 1). One SM's copy
+// engine serves several issue streams at once but one stream's copies one
+// after another, so two CTAs with two loader warps each keep four streams
+// going per SM; a single CTA with a ring twice as deep does as well on long
+// GEMMs.
 int env_int(const char* name, int dflt, int lo, int hi) {
   const char* e = std::getenv(name);
   if (e == nullptr) return dflt;
   const int v = std::atoi(e);
   return (v < lo || v > hi) ? dflt : v;
 }
-int ctas_per_sm() {
-  static const int v = env_int("SPENSE_CTAS_PER_SM", 2, 1, 2);
+// 0 (default) = automatic: one CTA per SM with a deep ring when the launch has
+// more row tiles than two-per-SM CTA slots (large GEMMs, stream-K) or more
+// than 32 tokens (the activation tile then fills half of every ring stage),
+// two per SM otherwise (short decode GEMMs, where a second CTA per SM hides
+// the fixed costs).
+int ctas_per_sm_knob() {
+  static const int v = env_int("SPENSE_CTAS_PER_SM", 0, 0, 2);
   return v;
 }
 // CTA slots per SM that one grid may fill (default: all of them); 1 leaves
@@ -208,7 +215,9 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.nsb > 0 ? 256u : 128u);
   pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.nsb > 0 ? kMetaBlockBytes : 0);
   const uint32_t reserve = 1024 + kBarrierBytes;  // alignment slack + barrier area
-  for (int cps = ctas_per_sm(); cps >= 1; --cps) {
+  const int cps_first =
+      ctas_per_sm_knob() != 0 ? ctas_per_sm_knob() : ((pl.tiles > 2 * sms || pl.npad > 32) ? 1 : 2);
+  for (int cps = cps_first; cps >= 1; --cps) {
     const uint32_t smem_budget = gemm_max_smem() / cps - (cps > 1 ? 1024u : 0u);
     const uint32_t tmem_budget = 512u / cps;
     const int stages = static_cast<int>(std::min<uint32_t>(kMaxStages, (smem_budget - reserve) / pl.stage_bytes));
