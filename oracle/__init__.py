@@ -54,6 +54,8 @@ def _load():
     lib.oracle_tile.restype = ctypes.c_int
     lib.oracle_gemm.argtypes = [P, P, I64, P, P, I64, I64, P, P, I64, P, P, ctypes.c_int]
     lib.oracle_gemm.restype = ctypes.c_int
+    lib.oracle_quantize.argtypes = [P, I64, I64, P, I64, P, P]
+    lib.oracle_quantize.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -162,6 +164,29 @@ def gemm(X, s_x, W, s_w, keep=None, rows=None, nthreads=None):
     if st != OR_OK:
         raise OracleError(st, "gemm")
     return y, b
+
+
+def quantize(X_bf16, dense_idx=None):
+    """Per-token FP8 quantisation of bf16 activations with the packed column
+    order fused in: s[m] = fp32(absmax / 448) (1 for a zero row), Xq[m][j] =
+    e4m3 round-to-nearest-even, saturating, of fp32(x[m][c(j)] / s[m]), where c
+    is sparse columns ascending then `dense_idx` (identity when None).
+    (Technical Summary §2B: the dense indices are permuted into a contiguous
+    block; the SlideSparse page, Activation Lifting: the rearrangement is
+    folded into per-token quantisation.)
+
+    X_bf16: uint16 bit patterns [M, K]. Returns (Xq uint8 [M, K], s float32 [M]).
+    """
+    X = np.ascontiguousarray(X_bf16, dtype=np.uint16)
+    M, K = X.shape
+    di = _idx(dense_idx)
+    Kd = 0 if di is None else di.shape[0]
+    Xq = np.zeros((M, K), np.uint8)
+    s = np.zeros(M, np.float32)
+    st = _load().oracle_quantize(_ptr(X), M, K, _ptr(di), Kd, _ptr(Xq), _ptr(s))
+    if st != OR_OK:
+        raise OracleError(st, "quantize")
+    return Xq, s
 
 
 def within_tolerance(y, yref, bound, rel=4e-3, absb=1e-5):

@@ -37,6 +37,10 @@
 //       restated here from their written definition (128-row tiles, 256
 //       compacted sparse columns or 128 dense columns per block, 128-byte
 //       swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)).
+//   R11 Per-token quantisation of the activations (the step in front of the
+//       GEMM) is computed in IEEE fp32: s = absmax / 448 (1 for an all-zero
+//       row), q = e4m3(x / s) rounded to nearest even and saturated to 448,
+//       one rounding per operation.
 //
 // Arithmetic: FP8 products and sums are accumulated in double precision.
 // Every e4m3 value is a dyadic rational with at most 4 significant bits, so
@@ -104,6 +108,35 @@ int build_order(int64_t K, const int32_t* dense_idx, int64_t Kd,
   for (int64_t k = 0; k < K; ++k)
     if (!is_dense[static_cast<size_t>(k)]) sparse_cols.push_back(k);
   return OR_OK;
+}
+
+// E4M3 encoding of a float by its definition: the finite code whose value is
+// nearest; on a tie the code with an even last bit (round to nearest, ties to
+// even); magnitudes above 448 saturate to 448; NaN gives 0x7F. The sign is
+// kept, so a negative value that rounds to zero gives 0x80.
+uint8_t encode_e4m3_rne_sat(float v) {
+  if (std::isnan(v)) return 0x7F;
+  const uint8_t sign = std::signbit(v) ? 0x80 : 0x00;
+  const double a = std::fabs(static_cast<double>(v));
+  if (a >= 448.0) return static_cast<uint8_t>(sign | 0x7E);
+  int best = 0;
+  double best_d = a;  // distance to code 0 (value 0)
+  for (int c = 1; c <= 0x7E; ++c) {
+    const double d = std::fabs(decode_e4m3(static_cast<uint8_t>(c)) - a);
+    if (d < best_d || (d == best_d && (c & 1) == 0)) {
+      best = c;
+      best_d = d;
+    }
+  }
+  return static_cast<uint8_t>(sign | best);
+}
+
+// bf16 bit pattern -> float (exact: bf16 is the upper half of a float).
+float bf16_to_float(uint16_t b) {
+  const uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return f;
 }
 
 }  // namespace
@@ -334,6 +367,47 @@ int oracle_gemm(const uint8_t* X, const float* s_x, int64_t M, const uint8_t* W,
       th.emplace_back(work, r0, r1);
     }
     for (auto& x : th) x.join();
+  }
+  return OR_OK;
+}
+
+
+// Per-token FP8 quantisation of bf16 activations, the step in front of the
+// GEMM, with the column rearrangement a scattered dense set needs fused in
+// (the SlideSparse page, "Activation Lifting", folds its rearrangement into
+// per-token quantisation the same way; the SpenseGPT page, 2.B, permutes the
+// dense indices into one contiguous block):
+//   s[m]    = fp32(max_k |x[m][k]| / 448), or 1 for an all-zero row
+//   q[m][j] = e4m3_rne_sat(fp32(x[m][c(j)] / s[m]))
+// where c is the column order sparse columns ascending then dense_idx
+// (dense_idx == NULL: the identity). Reading R11: the scale and each quotient
+// are single IEEE fp32 operations (one rounding each), the precision in which
+// the code of every element is decided.
+int oracle_quantize(const uint16_t* X, int64_t M, int64_t K, const int32_t* dense_idx, int64_t Kd,
+                    uint8_t* Xq, float* s) {
+  if (X == nullptr || Xq == nullptr || s == nullptr) return OR_ERR_ARG;
+  if (M < 0 || K < 0) return OR_ERR_SHAPE;
+  std::vector<int64_t> order(static_cast<size_t>(K));
+  if (dense_idx == nullptr) {
+    for (int64_t k = 0; k < K; ++k) order[static_cast<size_t>(k)] = k;
+  } else {
+    std::vector<int64_t> sp, dn;
+    const int st = build_order(K, dense_idx, Kd, sp, dn);
+    if (st != OR_OK) return st;
+    size_t j = 0;
+    for (int64_t k : sp) order[j++] = k;
+    for (int64_t k : dn) order[j++] = k;
+  }
+  for (int64_t m = 0; m < M; ++m) {
+    const uint16_t* xr = X + m * K;
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; ++k) amax = std::max(amax, std::fabs(bf16_to_float(xr[k])));
+    const float sm = amax > 0.0f ? amax / 448.0f : 1.0f;
+    s[m] = sm;
+    for (int64_t j = 0; j < K; ++j) {
+      const float q = bf16_to_float(xr[order[static_cast<size_t>(j)]]) / sm;
+      Xq[m * K + j] = encode_e4m3_rne_sat(q);
+    }
   }
   return OR_OK;
 }
