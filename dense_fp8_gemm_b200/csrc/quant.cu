@@ -1,0 +1,188 @@
+// Per-token FP8 quantisation of bf16 activations, with the column order of a
+// packed weight fused in.
+//
+// Pages: "SpenseGPT: Practical One-shot Pruning Enabling Sparse and Dense GEMMs
+// for LLM Inference" (gist.science technical summary), Technical Summary §2.B:
+// SpenseGPT+ keeps a scattered set of input indices dense and permutes them
+// into one contiguous block; the GEMM then needs the activations in that
+// column order. The SlideSparse page ("Activation Lifting") folds such a
+// rearrangement into the per-token quantisation that runs in front of every
+// FP8 GEMM anyway, at almost no extra cost. Here:
+//   s[m]    = fp32(max_k |x[m][k]| / 448)   (1 for an all-zero row)
+//   q[m][j] = e4m3 round-to-nearest-even, saturating, of fp32(x[m][c(j)] / s[m])
+// with c(j) = perm[j] (packed position -> original column) or j.
+//
+// DRAM sees each byte of X once: the repeated reads of a row (several CTAs per
+// row, and the quantising pass after the absmax pass) hit L2.
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "spense_internal.h"
+
+namespace spense {
+namespace {
+
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Two floats -> two e4m3 bytes (round to nearest even, saturating to +-448):
+// the low byte holds `lo`, the high byte `hi`.
+__device__ __forceinline__ uint16_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  float r = 0.0f;
+  for (int i = 0; i < kQuantThreads / 32; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+// Each row is split over C CTAs (C = 1 .. 8; more CTAs per row when there are
+// few rows). CTA c writes the 16-column output chunks [K16 c / C, K16 (c + 1) /
+// C) of the row. Every CTA reads the whole row to take its absmax itself (the
+// C - 1 extra reads of a row hit L2; no CTA waits for another), and with a
+// gather it keeps the row in shared memory and gathers from there. Rows too
+// long for shared memory gather from global memory instead (the packed order
+// is two ascending runs, so those loads mostly share cache lines).
+// K % 16 == 0; X rows 16-byte aligned; Xq rows 16-byte aligned.
+template <bool kGather, bool kStaged>
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t* __restrict__ X, int64_t K,
+                                                                 const int32_t* __restrict__ perm,
+                                                                 uint8_t* __restrict__ Xq, float* __restrict__ s_out,
+                                                                 int C) {
+  extern __shared__ uint4 qsmem[];  // kStaged: the row, K bf16
+  __shared__ float red[kQuantThreads / 32];
+  const int64_t m = blockIdx.x / C;
+  const int c = static_cast<int>(blockIdx.x % C);
+  const int64_t k16 = K / 16;
+  const int64_t j0 = k16 * c / C, j1 = k16 * (c + 1) / C;  // this CTA's 16-column chunks
+  const uint16_t* xrow = X + m * K;
+  const uint4* xr = reinterpret_cast<const uint4*>(xrow);
+  float amax = 0.0f;
+  // Absmax of the whole row: 16-byte loads, eight in flight per thread.
+  const int64_t n8 = K / 8;
+  for (int64_t i = threadIdx.x; i < n8; i += 8 * kQuantThreads) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int64_t ii = i + static_cast<int64_t>(u) * kQuantThreads;
+      v[u] = ii < n8 ? __ldg(xr + ii) : make_uint4(0u, 0u, 0u, 0u);
+      if (kStaged && ii < n8) qsmem[ii] = v[u];
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        amax = fmaxf(amax, fabsf(bf16_bits_to_float(w[h] & 0xFFFFu)));
+        amax = fmaxf(amax, fabsf(bf16_bits_to_float(w[h] >> 16)));
+      }
+    }
+  }
+  amax = block_max(amax, red);  // its barrier also publishes the staged row
+  const float s = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  if (c == 0 && threadIdx.x == 0) s_out[m] = s;
+  const uint16_t* src = kStaged ? reinterpret_cast<const uint16_t*>(qsmem) : xrow;
+  uint4* qr = reinterpret_cast<uint4*>(Xq + m * K);
+  // Four 16-column chunks per thread per round: all their loads are issued
+  // before any is used, so a round costs one memory latency, not four.
+  constexpr int kU = 4;
+  for (int64_t i0 = j0 + threadIdx.x; i0 < j1; i0 += kU * kQuantThreads) {
+    uint4 raw[kU][2];  // plain: the 16 bf16 of each chunk
+    int4 cs[kU][4];    // gather: the 16 source columns of each chunk
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = i0 + static_cast<int64_t>(u) * kQuantThreads;
+      if (i < j1) {
+        if (kGather) {
+          const int4* pj = reinterpret_cast<const int4*>(perm + i * 16);
+#pragma unroll
+          for (int h = 0; h < 4; ++h) cs[u][h] = __ldg(pj + h);
+        } else {
+          raw[u][0] = __ldg(xr + 2 * i);
+          raw[u][1] = __ldg(xr + 2 * i + 1);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int64_t i = i0 + static_cast<int64_t>(u) * kQuantThreads;
+      if (i >= j1) break;
+      float f[16];
+      if (kGather) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          f[4 * h + 0] = bf16_bits_to_float(kStaged ? src[cs[u][h].x] : __ldg(src + cs[u][h].x));
+          f[4 * h + 1] = bf16_bits_to_float(kStaged ? src[cs[u][h].y] : __ldg(src + cs[u][h].y));
+          f[4 * h + 2] = bf16_bits_to_float(kStaged ? src[cs[u][h].z] : __ldg(src + cs[u][h].z));
+          f[4 * h + 3] = bf16_bits_to_float(kStaged ? src[cs[u][h].w] : __ldg(src + cs[u][h].w));
+        }
+      } else {
+        const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                               raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          f[2 * h] = bf16_bits_to_float(w[h] & 0xFFFFu);
+          f[2 * h + 1] = bf16_bits_to_float(w[h] >> 16);
+        }
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f[4 * h], s), __fdiv_rn(f[4 * h + 1], s));
+        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f[4 * h + 2], s), __fdiv_rn(f[4 * h + 3], s));
+        o[h] = lo | (hi << 16);
+      }
+      qr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+}
+
+// Shared memory for a staged row: at most 56 KB, so four CTAs fit per SM.
+constexpr int64_t kQuantStageBytes = 56 * 1024;
+
+}  // namespace
+
+cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, uint8_t* Xq,
+                            float* s_x, int sms, cudaStream_t stream) {
+  if (M == 0) return cudaSuccess;
+  // CTAs per row: one once the rows alone cover the SMs (every extra CTA of a
+  // row reads the row again); otherwise enough for two CTAs per SM, at most 8
+  // and at most one per 16-column chunk.
+  int64_t C = M >= sms ? 1 : (2 * static_cast<int64_t>(sms) + M - 1) / M;
+  C = C < 1 ? 1 : (C > 8 ? 8 : C);
+  while (C > 1 && K / 16 < C) --C;
+  const unsigned int grid = static_cast<unsigned int>(M * C);
+  const int ci = static_cast<int>(C);
+  if (perm == nullptr) {
+    quantize_kernel<false, false><<<grid, kQuantThreads, 0, stream>>>(X, K, perm, Xq, s_x, ci);
+    return cudaGetLastError();
+  }
+  const int64_t stage = K * 2;
+  if (stage > kQuantStageBytes) {
+    quantize_kernel<true, false><<<grid, kQuantThreads, 0, stream>>>(X, K, perm, Xq, s_x, ci);
+    return cudaGetLastError();
+  }
+  static thread_local int configured_for = -1;
+  int dev = 0;
+  cudaError_t st = cudaGetDevice(&dev);
+  if (st != cudaSuccess) return st;
+  if (configured_for != dev) {
+    st = cudaFuncSetAttribute(quantize_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kQuantStageBytes));
+    if (st != cudaSuccess) return st;
+    configured_for = dev;
+  }
+  quantize_kernel<true, true><<<grid, kQuantThreads, static_cast<size_t>(stage), stream>>>(X, K, perm, Xq, s_x, ci);
+  return cudaGetLastError();
+}
+
+}  // namespace spense

@@ -333,10 +333,11 @@ spense_status check_gemm_args(const spense_packed* const* hs, int count, int64_t
 
 // Enqueue one launch over `count` packed weights sharing X (arguments validated).
 spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t* X, const float* x_scale,
-                       int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream) {
+                       int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream,
+                       bool x_packed_order = false) {
   const spense_packed* h0 = hs[0];
   const uint8_t* xsrc = X;
-  if (h0->perm != nullptr) {
+  if (h0->perm != nullptr && !x_packed_order) {
     uint8_t* xg = ws + pl.ws.xg_off;
     cudaError_t e = launch_gather(X, h0->perm, M, h0->K, xg, stream);
     if (e != cudaSuccess) return cuda_fail(e, "gather launch");
@@ -564,6 +565,14 @@ size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M) {
 spense_status spense_gemm_grouped(const spense_packed* const* Wps, int count, const uint8_t* X,
                                   const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
                                   size_t workspace_bytes, void* stream_v) {
+  return spense_gemm_grouped_ex(Wps, count, X, x_scale, M, Ys, workspace, workspace_bytes, 0u, stream_v);
+}
+
+spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count, const uint8_t* X,
+                                     const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
+                                     size_t workspace_bytes, unsigned int flags, void* stream_v) {
+  if ((flags & ~static_cast<unsigned int>(SPENSE_GEMM_X_PACKED_ORDER)) != 0u)
+    return fail(SPENSE_ERR_ARG, "unknown flags %#x", flags);
   if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
   if (X == nullptr || x_scale == nullptr || Ys == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
   if (!aligned(X, 16) || !aligned(x_scale, 4))
@@ -584,8 +593,34 @@ spense_status spense_gemm_grouped(const spense_packed* const* Wps, int count, co
     return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
                 pl.ws.total_device);
   st = run_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
-                static_cast<cudaStream_t>(stream_v));
+                static_cast<cudaStream_t>(stream_v), (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u);
   return st == SPENSE_OK ? ok() : st;
+}
+
+spense_status spense_quantize(const uint16_t* X, int64_t M, int64_t K, const spense_packed* order, uint8_t* Xq,
+                              float* x_scale, void* stream_v) {
+  if (M < 0 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [0, 65535]", (long long)M);
+  if (M > 0 && (X == nullptr || Xq == nullptr || x_scale == nullptr))
+    return fail(SPENSE_ERR_ARG, "X, Xq or x_scale is NULL");
+  if (K < 16 || K > (1 << 20) || K % 16 != 0)
+    return fail(SPENSE_ERR_SHAPE, "K = %lld must be a positive multiple of 16 up to 2^20", (long long)K);
+  if (!aligned(X, 16) || !aligned(Xq, 16) || !aligned(x_scale, 4))
+    return fail(SPENSE_ERR_ALIGN, "X and Xq must be 16-byte aligned, x_scale 4-byte aligned");
+  const int32_t* perm = nullptr;
+  if (order != nullptr) {
+    if (order->K != K) return fail(SPENSE_ERR_SHAPE, "order was packed with K = %lld, not %lld",
+                                   (long long)order->K, (long long)K);
+    perm = order->perm;  // NULL for a tail dense set: the packed order is the identity
+  }
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  if (order != nullptr && dev != order->device)
+    return fail(SPENSE_ERR_ARG, "order was packed on device %d, current device is %d", order->device, dev);
+  cudaError_t e = launch_quantize(X, M, K, perm, Xq, x_scale, info.sms, static_cast<cudaStream_t>(stream_v));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return ok();
 }
 
 spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale, int64_t M,

@@ -104,6 +104,8 @@ cudaError_t launch_gather(const uint8_t* X, const int32_t* perm, int64_t M, int6
 cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t smem_bytes,
                         cudaStream_t stream);
 uint32_t gemm_max_smem();
+cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, uint8_t* Xq,
+                            float* s_x, int sms, cudaStream_t stream);
 
 // Device error bits written by the pack kernel.
 constexpr unsigned int kPackErrMask = 1u;

@@ -28,8 +28,10 @@ SYMBOLS = (
     "spense_pack", "spense_gemm", "spense_gemm_workspace_size", "spense_gemm_host",
     "spense_gemm_host_workspace_size", "spense_free", "spense_get_info",
     "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
-    "spense_gemm_grouped", "spense_gemm_grouped_workspace_size",
+    "spense_gemm_grouped", "spense_gemm_grouped_workspace_size", "spense_gemm_grouped_ex",
+    "spense_quantize",
 )
+GEMM_X_PACKED_ORDER = 1
 MAX_GROUP = 4
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -76,6 +78,9 @@ def lib() -> ctypes.CDLL:
     L.spense_gemm_grouped.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ, P]
     L.spense_gemm_grouped_workspace_size.argtypes = [ctypes.POINTER(P), ctypes.c_int, I64]
     L.spense_gemm_grouped_workspace_size.restype = SZ
+    L.spense_gemm_grouped_ex.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ,
+                                         U32, P]
+    L.spense_quantize.argtypes = [P, I64, I64, P, P, P, P]
     L.spense_last_error.restype = ctypes.c_char_p
     L.spense_version.restype = ctypes.c_char_p
     for name in ("spense_pack", "spense_gemm", "spense_gemm_host", "spense_free", "spense_get_info",
@@ -266,9 +271,11 @@ def grouped_workspace_size(pws, M: int) -> int:
 
 
 def gemm_grouped(pws, X: torch.Tensor, x_scale: torch.Tensor, Ys=None, workspace: torch.Tensor | None = None,
-                 stream=None):
-    """spense_gemm_grouped: one launch over several packed weights sharing X
-    (same K, Kd and dense column set). Returns the list of outputs."""
+                 stream=None, flags: int = 0):
+    """spense_gemm_grouped (flags == 0) or spense_gemm_grouped_ex: one launch
+    over several packed weights sharing X (same K, Kd and dense column set).
+    flags = GEMM_X_PACKED_ORDER: X is already in the packed column order (from
+    quantize(..., order=pw)). Returns the list of outputs."""
     M = X.shape[0]
     if Ys is None:
         Ys = [torch.empty((M, pw.N), dtype=torch.bfloat16, device=X.device) for pw in pws]
@@ -277,12 +284,31 @@ def gemm_grouped(pws, X: torch.Tensor, x_scale: torch.Tensor, Ys=None, workspace
     yarr = (ctypes.c_void_p * len(pws))()
     for i, Y in enumerate(Ys):
         yarr[i] = _dev_ptr(Y, torch.bfloat16, f"Y[{i}]").value
-    code = lib().spense_gemm_grouped(_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"),
-                                     _dev_ptr(x_scale, torch.float32, "x_scale"), M, yarr,
-                                     _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
-                                     _stream(stream))
-    _check(code, "spense_gemm_grouped")
+    args = (_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"), _dev_ptr(x_scale, torch.float32, "x_scale"),
+            M, yarr, _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel())
+    if flags == 0:
+        _check(lib().spense_gemm_grouped(*args, _stream(stream)), "spense_gemm_grouped")
+    else:
+        _check(lib().spense_gemm_grouped_ex(*args, int(flags), _stream(stream)), "spense_gemm_grouped_ex")
     return Ys
+
+
+def quantize(X: torch.Tensor, order: PackedWeight | None = None, Xq: torch.Tensor | None = None,
+             x_scale: torch.Tensor | None = None, stream=None):
+    """spense_quantize: per-token FP8 quantisation of bf16 activations X [M, K]
+    (s = absmax / 448 in fp32, e4m3 round-to-nearest-even, saturating), with the
+    columns in `order`'s packed order when a packed weight is given. Returns
+    (Xq uint8 [M, K], x_scale float32 [M])."""
+    M, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.uint8, device=X.device)
+    if x_scale is None:
+        x_scale = torch.empty((M,), dtype=torch.float32, device=X.device)
+    code = lib().spense_quantize(_dev_ptr(X, torch.bfloat16, "X"), M, K, None if order is None else order.handle,
+                                 _dev_ptr(Xq, torch.uint8, "Xq"), _dev_ptr(x_scale, torch.float32, "x_scale"),
+                                 _stream(stream))
+    _check(code, "spense_quantize")
+    return Xq, x_scale
 
 
 def gemm_noalloc(pw: PackedWeight, X: torch.Tensor, x_scale: torch.Tensor, Y: torch.Tensor,

@@ -159,6 +159,53 @@ SPENSE_API spense_status spense_gemm_grouped(const spense_packed* const* Wps, in
 
 SPENSE_API size_t spense_gemm_grouped_workspace_size(const spense_packed* const* Wps, int count, int64_t M);
 
+/* Flags of spense_gemm_grouped_ex. */
+enum {
+  /* X (and x_scale) are already in the packed column order of the weights
+   * (sparse columns ascending, then the dense columns in dense_idx order), as
+   * spense_quantize writes them when given one of the weights as `order`; the
+   * GEMM then skips its own gather. No effect for a tail dense set. */
+  SPENSE_GEMM_X_PACKED_ORDER = 1u
+};
+
+/*
+ * spense_gemm_grouped_ex — spense_gemm_grouped with flags (above); unknown
+ * flag bits are an ARG error. With flags == 0 it is spense_gemm_grouped.
+ */
+SPENSE_API spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count, const uint8_t* X,
+                                                const float* x_scale, int64_t M, uint16_t* const* Ys,
+                                                void* workspace, size_t workspace_bytes, unsigned int flags,
+                                                void* stream);
+
+/*
+ * spense_quantize — per-token FP8 quantisation of bf16 activations, the step in
+ * front of every FP8 GEMM, with the column order of a packed weight fused in.
+ * The technical summary of "SpenseGPT: Practical One-shot Pruning Enabling
+ * Sparse and Dense GEMMs for LLM Inference" (§2.B) permutes SpenseGPT+'s
+ * scattered dense indices into one contiguous block, so the GEMM reads the
+ * activations in that order; the SlideSparse page ("Activation Lifting") folds
+ * such a rearrangement into the per-token quantisation at almost no cost. This
+ * does the same, so the GEMM's own gather can be skipped
+ * (SPENSE_GEMM_X_PACKED_ORDER).
+ *   X        device, bf16 bit patterns [M][K] row-major, 16-byte aligned.
+ *   M        0 .. 65535 token rows (0: nothing to do).
+ *   K        multiple of 16, 16 .. 2^20.
+ *   order    NULL: columns stay in X's order. A packed weight with the same K on
+ *            the current device: columns come out in its packed order (the
+ *            identity for a tail dense set).
+ *   Xq       device, e4m3 [M][K] row-major, 16-byte aligned (caller-owned).
+ *   x_scale  device, fp32 [M], 4-byte aligned (caller-owned).
+ * Result, in IEEE fp32 with one rounding per operation:
+ *   x_scale[m] = max_k |X[m][k]| / 448 (1 for an all-zero row)
+ *   Xq[m][j]   = e4m3 round-to-nearest-even of X[m][c(j)] / x_scale[m],
+ *                saturated to +-448 (c = the packed order or the identity).
+ * X must be finite; a NaN or infinity gives unspecified codes for its row.
+ * Asynchronous on `stream`. Errors: ARG (NULL pointer, order from another
+ * device), SHAPE, ALIGN, UNSUPPORTED (no sm_100 device), CUDA.
+ */
+SPENSE_API spense_status spense_quantize(const uint16_t* X, int64_t M, int64_t K, const spense_packed* order,
+                                         uint8_t* Xq, float* x_scale, void* stream);
+
 /*
  * spense_gemm_host — the same GEMM on HOST buffers: copies X [M][K] and
  * x_scale [M] from host memory into the workspace, runs spense_gemm, copies Y

@@ -116,3 +116,38 @@ def test_valid_arguments_without_a_device_report_unsupported(L):
         pytest.skip("a GPU is present")
     code, out = _pack_raw(L)
     assert code == 11 and out.value is None
+
+
+def _quant_raw(L, X=0x1000, M=4, K=256, order=None, Xq=0x8000, s=0x9000):
+    v = lambda a: ctypes.c_void_p(a) if a else None
+    return L.spense_quantize(v(X), M, K, v(order), v(Xq), v(s), None)
+
+
+def test_quantize_rejects_bad_arguments(L):
+    assert _quant_raw(L, X=0) == 1
+    assert _quant_raw(L, Xq=0) == 1
+    assert _quant_raw(L, s=0) == 1
+    for M, K in [(-1, 256), (65536, 256), (4, 8), (4, 264 - 4), (4, 0), (4, (1 << 20) + 16)]:
+        assert _quant_raw(L, M=M, K=K) == 2, (M, K)
+    assert _quant_raw(L, X=0x1008) == 3
+    assert _quant_raw(L, Xq=0x8004) == 3
+    assert _quant_raw(L, s=0x9002) == 3
+
+
+def test_gemm_ex_rejects_unknown_flags(L):
+    h = (ctypes.c_void_p * 1)(0x10)
+    y = (ctypes.c_void_p * 1)(0x3000)
+    code = L.spense_gemm_grouped_ex(h, 1, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 1, y,
+                                    ctypes.c_void_p(0x4000), 1 << 20, 0x2, None)
+    assert code == 1 and b"flags" in L.spense_last_error()
+
+
+def test_quantize_without_a_device_reports_unsupported(L):
+    try:
+        import torch
+        has_gpu = torch.cuda.is_available()
+    except Exception:
+        has_gpu = False
+    if has_gpu:
+        pytest.skip("a GPU is present")
+    assert _quant_raw(L) == 11
