@@ -56,6 +56,10 @@ def _load():
     lib.oracle_gemm.restype = ctypes.c_int
     lib.oracle_quantize.argtypes = [P, I64, I64, P, I64, P, P]
     lib.oracle_quantize.restype = ctypes.c_int
+    lib.oracle_score_glu.argtypes = [P, P, P, P, I64, I64, P, P, P, P, P]
+    lib.oracle_score_glu.restype = ctypes.c_int
+    lib.oracle_select_top.argtypes = [P, I64, I64, P]
+    lib.oracle_select_top.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -187,6 +191,34 @@ def quantize(X_bf16, dense_idx=None):
     if st != OR_OK:
         raise OracleError(st, "quantize")
     return Xq, s
+
+
+def score_glu(down, s_down, h_in, h_mid, gate=None, s_gate=None, up=None, s_up=None):
+    """SpenseGPT+ importance of every intermediate index of a GLU MLP, float64
+    (Technical Summary §2B: S_ij = |W_ij| sqrt(H_jj) aggregated over gate, up
+    and down). gate/up: e4m3 [I, H] with fp32 row scales [I]; down: e4m3 [H, I]
+    with row scales [H]; h_in [H], h_mid [I]: Hessian diagonals. Returns [I]."""
+    down = _u8(down)
+    H, I = down.shape
+    f32 = lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.float32)
+    g, u = _u8(gate), _u8(up)
+    out = np.zeros(I, np.float64)
+    st = _load().oracle_score_glu(_ptr(g), _ptr(f32(s_gate)), _ptr(u), _ptr(f32(s_up)), I, H, _ptr(down),
+                                  _ptr(f32(s_down)), _ptr(f32(h_in)), _ptr(f32(h_mid)), _ptr(out))
+    if st != OR_OK:
+        raise OracleError(st, "score_glu")
+    return out
+
+
+def select_top(score, Kd):
+    """The Kd largest scores (ties to the lower index), ascending indices
+    (Technical Summary §2B: the top-scoring indices stay dense)."""
+    sc = np.ascontiguousarray(score, dtype=np.float64)
+    out = np.zeros(Kd, np.int32)
+    st = _load().oracle_select_top(_ptr(sc), sc.shape[0], int(Kd), _ptr(out))
+    if st != OR_OK:
+        raise OracleError(st, "select_top")
+    return out
 
 
 def within_tolerance(y, yref, bound, rel=4e-3, absb=1e-5):

@@ -37,6 +37,15 @@
 //       restated here from their written definition (128-row tiles, 256
 //       compacted sparse columns or 128 dense columns per block, 128-byte
 //       swizzle: 16-byte chunk c of row r sits at chunk c ^ (r & 7)).
+//   R12 SpenseGPT+ importance of intermediate index t of a GLU MLP (gate and
+//       up [I][H], down [H][I]; weights are e4m3 codes times their fp32 row
+//       scales; h_in [H] and h_mid [I] are the diagonals of the input Hessians
+//       of gate/up and of down): the Wanda terms |W_ij| sqrt(H_jj) of every
+//       weight that touches t, summed:
+//         score[t] = sum_j |gate[t][j]| sqrt(h_in[j]) + sum_j |up[t][j]| sqrt(h_in[j])
+//                  + sqrt(h_mid[t]) sum_i |down[i][t]|
+//       The Kd indices with the largest scores stay dense (ties to the lower
+//       index), listed in ascending order.
 //   R11 Per-token quantisation of the activations (the step in front of the
 //       GEMM) is computed in IEEE fp32: s = absmax / 448 (1 for an all-zero
 //       row), q = e4m3(x / s) rounded to nearest even and saturated to 448,
@@ -409,6 +418,53 @@ int oracle_quantize(const uint16_t* X, int64_t M, int64_t K, const int32_t* dens
       Xq[m * K + j] = encode_e4m3_rne_sat(q);
     }
   }
+  return OR_OK;
+}
+
+
+// SpenseGPT+ importance scores (the SpenseGPT page, 2.B: a Wanda-style score
+// S_ij = |W_ij| sqrt(H_jj) aggregated over the gate, up and down projections;
+// reading R12). gate or up may be NULL (its term is left out). double precision.
+int oracle_score_glu(const uint8_t* gate, const float* s_gate, const uint8_t* up, const float* s_up,
+                     int64_t I, int64_t H, const uint8_t* down, const float* s_down, const float* h_in,
+                     const float* h_mid, double* score) {
+  if (down == nullptr || s_down == nullptr || h_in == nullptr || h_mid == nullptr || score == nullptr)
+    return OR_ERR_ARG;
+  if ((gate != nullptr && s_gate == nullptr) || (up != nullptr && s_up == nullptr)) return OR_ERR_ARG;
+  if (I < 0 || H < 0) return OR_ERR_SHAPE;
+  double table[256];
+  oracle_e4m3_table(table);
+  for (int64_t t = 0; t < I; ++t) {
+    double total = 0.0;
+    for (int w = 0; w < 2; ++w) {
+      const uint8_t* Wm = w == 0 ? gate : up;
+      const float* sc = w == 0 ? s_gate : s_up;
+      if (Wm == nullptr) continue;
+      double acc = 0.0;
+      for (int64_t j = 0; j < H; ++j)
+        acc += std::fabs(static_cast<double>(sc[t]) * table[Wm[t * H + j]]) * std::sqrt(static_cast<double>(h_in[j]));
+      total += acc;
+    }
+    double col = 0.0;
+    for (int64_t i = 0; i < H; ++i) col += std::fabs(static_cast<double>(s_down[i]) * table[down[i * I + t]]);
+    total += std::sqrt(static_cast<double>(h_mid[t])) * col;
+    score[t] = total;
+  }
+  return OR_OK;
+}
+
+// The Kd largest scores (ties to the lower index), written in ascending index
+// order: the dense set SpenseGPT+ keeps (the SpenseGPT page, 2.B: "the
+// top-scoring indices are selected to remain dense").
+int oracle_select_top(const double* score, int64_t I, int64_t Kd, int32_t* out) {
+  if (score == nullptr || (Kd > 0 && out == nullptr)) return OR_ERR_ARG;
+  if (I < 0 || Kd < 0 || Kd > I) return OR_ERR_SHAPE;
+  std::vector<int64_t> idx(static_cast<size_t>(I));
+  for (int64_t t = 0; t < I; ++t) idx[static_cast<size_t>(t)] = t;
+  std::stable_sort(idx.begin(), idx.end(), [&](int64_t a, int64_t b) { return score[a] > score[b]; });
+  std::vector<int64_t> top(idx.begin(), idx.begin() + Kd);
+  std::sort(top.begin(), top.end());
+  for (int64_t j = 0; j < Kd; ++j) out[j] = static_cast<int32_t>(top[static_cast<size_t>(j)]);
   return OR_OK;
 }
 
