@@ -44,9 +44,10 @@ def parse():
     ap.add_argument("--dense-frac", type=float, default=0.25)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["gemm", "quantize"], default="gemm",
+    ap.add_argument("--op", choices=["gemm", "quantize", "score"], default="gemm",
                     help="gemm: the hybrid GEMM (default, the headline); quantize: the per-token FP8 "
-                         "quantisation with the SpenseGPT+ column order fused in")
+                         "quantisation with the SpenseGPT+ column order fused in; score: the SpenseGPT+ "
+                         "dense-set scorer and top-Kd selection")
     return ap.parse_args()
 
 
@@ -581,12 +582,89 @@ def run_quantize(args):
     return 0
 
 
+def run_score(args):
+    """SpenseGPT+ dense-set selection on the 32B-class FFN shapes: scores of the
+    I = 25600 intermediate indices from gate, up [I][5120] and down [5120][I]
+    (FP8 + row scales, synthetic Hessian diagonals), then the top Kd = 0.25 I.
+    One step = score + select. HBM roofline over the algorithmic bytes (the
+    three weight matrices, their scales, the Hessian diagonals, the scores)."""
+    import torch
+    from dense_fp8_gemm_b200 import spense, synth
+    import oracle
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    I, H = 25600, 5120
+    Kd = int(round(args.dense_frac * I))
+    g = np.random.default_rng(2)
+    sets = []
+    copies = 2  # 2 x 393 MB of weights, larger than L2
+    for c in range(copies):
+        gq, gs = synth.quantize_rows(synth.normal(2, 10 + c, (I, H), 0.02))
+        uq, us = synth.quantize_rows(synth.normal(2, 20 + c, (I, H), 0.02))
+        dq, ds = synth.quantize_rows(synth.normal(2, 30 + c, (H, I), 0.02))
+        sets.append({k: torch.from_numpy(v).to(dev) for k, v in
+                     dict(gate=gq, s_gate=gs, up=uq, s_up=us, down=dq, s_down=ds).items()})
+    h_in = torch.from_numpy((g.standard_normal((8, H)).astype(np.float32) ** 2).sum(0)).to(dev)
+    h_mid = torch.from_numpy((g.standard_normal((8, I)).astype(np.float32) ** 2).sum(0)).to(dev)
+    score = torch.empty((I,), dtype=torch.float32, device=dev)
+    idx = torch.empty((Kd,), dtype=torch.int32, device=dev)
+    ws = spense.new_workspace(max(256, int(spense.lib().spense_score_workspace_size(I, H))), dev)
+    bytes_per = 3 * I * H + 4 * (2 * I + H) + 4 * (H + I) + 4 * I + 4 * Kd
+
+    def launch(i, st):
+        w = sets[i]
+        spense.score_glu(w["down"], w["s_down"], h_in, h_mid, gate=w["gate"], s_gate=w["s_gate"], up=w["up"],
+                         s_up=w["s_up"], score=score, workspace=ws, stream=st)
+        spense.select_dense(score, Kd, out=idx, stream=st)
+
+    steps = max(20, min(args.steps // 100, 200))
+    with ClockSampler(0) as clocks:
+        t0w = time.time()
+        t_step, n = graph_time(launch, copies, steps, args.warmup // 20)
+        clocks.mark(t0w, time.time())
+    peak, peak_kind = read_peaks()
+    cpu = None
+    if not args.no_cpu_baseline:
+        w = {k: v.cpu().numpy() for k, v in sets[0].items()}
+        cols = 512  # a bounded sample: the scores of 512 intermediate indices
+        sub = dict(gate=w["gate"][:cols], s_gate=w["s_gate"][:cols], up=w["up"][:cols], s_up=w["s_up"][:cols],
+                   down=np.ascontiguousarray(w["down"][:, :cols]), s_down=w["s_down"])
+        hi, hm = h_in.cpu().numpy(), h_mid.cpu().numpy()[:cols]
+        c0, done = time.time(), 0
+        while time.time() - c0 < min(args.cpu_seconds, 5.0) or done == 0:
+            oracle.score_glu(sub["down"], sub["s_down"], hi, hm, gate=sub["gate"], s_gate=sub["s_gate"],
+                             up=sub["up"], s_up=sub["s_up"])
+            done += 1
+        el = time.time() - c0
+        cpu = {"value": done * 3 * cols * H / el / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"scores of {cols} of {I} intermediate indices (weight bytes only), {done} passes in "
+                         f"{el:.1f} s"}
+    line = {
+        "metric": "spense_score_select_GBps", "value": bytes_per / t_step / 1e9, "unit": "GB/s", "n_gpus": 1,
+        "steps": n, "warmup": args.warmup // 20, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3->f32", "data": "synthetic",
+        "config": {"workload": f"SpenseGPT+ dense-set selection, 32B FFN: gate/up {I}x{H}, down {H}x{I}, "
+                               f"Kd = {Kd}", "l2": f"{copies} weight sets rotated (786 MB, larger than L2)"},
+        "roofline": {"bound": "hbm", "achieved": bytes_per / t_step / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": bytes_per / t_step / 1e9 / peak, "traffic": None, "peak_source": peak_kind,
+                     "kernel": "score_rows + score_cols + score_finish + select_top", "bytes_per_step": bytes_per},
+        "cpu_baseline": cpu,
+        "e2e": None,
+        "gpu_launches": n * 4,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
     if args.op == "quantize":
         return run_quantize(args)
+    if args.op == "score":
+        return run_score(args)
     return run_spense(args)
 
 

@@ -623,6 +623,55 @@ spense_status spense_quantize(const uint16_t* X, int64_t M, int64_t K, const spe
   return ok();
 }
 
+size_t spense_score_workspace_size(int64_t I, int64_t H) {
+  if (I < 16 || I > (1 << 20) || I % 16 != 0 || H < 16 || H > (1 << 20) || H % 16 != 0) return 0;
+  return score_workspace_bytes(I);
+}
+
+spense_status spense_score_glu(const uint8_t* gate, const float* s_gate, const uint8_t* up, const float* s_up,
+                               int64_t I, int64_t H, const uint8_t* down, const float* s_down, const float* h_in,
+                               const float* h_mid, float* score, void* workspace, size_t workspace_bytes,
+                               void* stream_v) {
+  if (down == nullptr || s_down == nullptr || h_in == nullptr || h_mid == nullptr || score == nullptr)
+    return fail(SPENSE_ERR_ARG, "down, s_down, h_in, h_mid or score is NULL");
+  if ((gate != nullptr && s_gate == nullptr) || (up != nullptr && s_up == nullptr))
+    return fail(SPENSE_ERR_ARG, "gate or up given without its row scales");
+  if (I < 16 || I > (1 << 20) || I % 16 != 0 || H < 16 || H > (1 << 20) || H % 16 != 0)
+    return fail(SPENSE_ERR_SHAPE, "I = %lld and H = %lld must be multiples of 16 in [16, 2^20]", (long long)I,
+                (long long)H);
+  if (!aligned(down, 16) || (gate && !aligned(gate, 16)) || (up && !aligned(up, 16)) || !aligned(s_down, 4) ||
+      (s_gate && !aligned(s_gate, 4)) || (s_up && !aligned(s_up, 4)) || !aligned(h_in, 4) || !aligned(h_mid, 4) ||
+      !aligned(score, 4))
+    return fail(SPENSE_ERR_ALIGN, "weights must be 16-byte aligned, vectors 4-byte aligned");
+  if (workspace == nullptr || workspace_bytes < score_workspace_bytes(I))
+    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                score_workspace_bytes(I));
+  if (!aligned(workspace, 256)) return fail(SPENSE_ERR_ALIGN, "workspace is not 256-byte aligned");
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  cudaError_t e = launch_score_glu(gate, s_gate, up, s_up, I, H, down, s_down, h_in, h_mid, score,
+                                   static_cast<float*>(workspace), static_cast<cudaStream_t>(stream_v));
+  if (e != cudaSuccess) return cuda_fail(e, "score launch");
+  return ok();
+}
+
+spense_status spense_select_dense(const float* score, int64_t I, int64_t Kd, int32_t* dense_idx, void* stream_v) {
+  if (I < 1 || I > (1 << 20)) return fail(SPENSE_ERR_SHAPE, "I = %lld outside [1, 2^20]", (long long)I);
+  if (Kd < 0 || Kd > I) return fail(SPENSE_ERR_SHAPE, "Kd = %lld outside [0, I]", (long long)Kd);
+  if (Kd > 0 && (score == nullptr || dense_idx == nullptr)) return fail(SPENSE_ERR_ARG, "score or dense_idx is NULL");
+  if (Kd > 0 && (!aligned(score, 4) || !aligned(dense_idx, 4)))
+    return fail(SPENSE_ERR_ALIGN, "score and dense_idx must be 4-byte aligned");
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  cudaError_t e = launch_select_top(score, I, Kd, dense_idx, static_cast<cudaStream_t>(stream_v));
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  return ok();
+}
+
 spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, const float* x_scale, int64_t M,
                           uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream_v) {
   if (Y == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");

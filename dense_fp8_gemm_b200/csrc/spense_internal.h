@@ -104,6 +104,11 @@ cudaError_t launch_gather(const uint8_t* X, const int32_t* perm, int64_t M, int6
 cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t smem_bytes,
                         cudaStream_t stream);
 uint32_t gemm_max_smem();
+size_t score_workspace_bytes(int64_t I);
+cudaError_t launch_score_glu(const uint8_t* gate, const float* s_gate, const uint8_t* up, const float* s_up,
+                             int64_t I, int64_t H, const uint8_t* down, const float* s_down, const float* h_in,
+                             const float* h_mid, float* score, float* partial, cudaStream_t stream);
+cudaError_t launch_select_top(const float* score, int64_t I, int64_t Kd, int32_t* out, cudaStream_t stream);
 cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32_t* perm, uint8_t* Xq,
                             float* s_x, int sms, cudaStream_t stream);
 

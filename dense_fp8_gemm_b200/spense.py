@@ -29,7 +29,7 @@ SYMBOLS = (
     "spense_gemm_host_workspace_size", "spense_free", "spense_get_info",
     "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
     "spense_gemm_grouped", "spense_gemm_grouped_workspace_size", "spense_gemm_grouped_ex",
-    "spense_quantize",
+    "spense_quantize", "spense_score_glu", "spense_score_workspace_size", "spense_select_dense",
 )
 GEMM_X_PACKED_ORDER = 1
 MAX_GROUP = 4
@@ -81,6 +81,10 @@ def lib() -> ctypes.CDLL:
     L.spense_gemm_grouped_ex.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ,
                                          U32, P]
     L.spense_quantize.argtypes = [P, I64, I64, P, P, P, P]
+    L.spense_score_glu.argtypes = [P, P, P, P, I64, I64, P, P, P, P, P, P, SZ, P]
+    L.spense_score_workspace_size.argtypes = [I64, I64]
+    L.spense_score_workspace_size.restype = SZ
+    L.spense_select_dense.argtypes = [P, I64, I64, P, P]
     L.spense_last_error.restype = ctypes.c_char_p
     L.spense_version.restype = ctypes.c_char_p
     for name in ("spense_pack", "spense_gemm", "spense_gemm_host", "spense_free", "spense_get_info",
@@ -334,3 +338,38 @@ def workspace_status(workspace: torch.Tensor, stream=None) -> int:
 
 def version() -> str:
     return lib().spense_version().decode()
+
+
+def score_glu(down: torch.Tensor, s_down: torch.Tensor, h_in: torch.Tensor, h_mid: torch.Tensor,
+              gate: torch.Tensor | None = None, s_gate: torch.Tensor | None = None,
+              up: torch.Tensor | None = None, s_up: torch.Tensor | None = None,
+              score: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """spense_score_glu: SpenseGPT+ importance of every intermediate index of a
+    GLU MLP. gate/up: uint8 e4m3 [I, H] (+ fp32 row scales [I]); down: uint8 e4m3
+    [H, I] (+ fp32 [H]); h_in [H], h_mid [I] fp32 Hessian diagonals. Returns
+    score fp32 [I]."""
+    H, I = down.shape
+    if score is None:
+        score = torch.empty((I,), dtype=torch.float32, device=down.device)
+    if workspace is None:
+        workspace = new_workspace(max(256, int(lib().spense_score_workspace_size(I, H))), down.device)
+    code = lib().spense_score_glu(_dev_ptr(gate, torch.uint8, "gate"), _dev_ptr(s_gate, torch.float32, "s_gate"),
+                                  _dev_ptr(up, torch.uint8, "up"), _dev_ptr(s_up, torch.float32, "s_up"), I, H,
+                                  _dev_ptr(down, torch.uint8, "down"), _dev_ptr(s_down, torch.float32, "s_down"),
+                                  _dev_ptr(h_in, torch.float32, "h_in"), _dev_ptr(h_mid, torch.float32, "h_mid"),
+                                  _dev_ptr(score, torch.float32, "score"),
+                                  _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    _check(code, "spense_score_glu")
+    return score
+
+
+def select_dense(score: torch.Tensor, Kd: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """spense_select_dense: the Kd largest scores (ties to the lower index) as
+    ascending int32 indices on the device."""
+    I = score.shape[0]
+    if out is None:
+        out = torch.empty((Kd,), dtype=torch.int32, device=score.device)
+    code = lib().spense_select_dense(_dev_ptr(score, torch.float32, "score"), I, int(Kd),
+                                     _dev_ptr(out, torch.int32, "dense_idx") if Kd > 0 else None, _stream(stream))
+    _check(code, "spense_select_dense")
+    return out

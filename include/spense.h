@@ -207,6 +207,49 @@ SPENSE_API spense_status spense_quantize(const uint16_t* X, int64_t M, int64_t K
                                          uint8_t* Xq, float* x_scale, void* stream);
 
 /*
+ * spense_score_glu — SpenseGPT+ importance of every intermediate index of a
+ * GLU MLP (Technical Summary §2.B: a Wanda-style score S_ij = |W_ij| sqrt(H_jj)
+ * aggregated across the gate, up and down projections; the top-scoring indices
+ * stay dense). This library's reading of the aggregation, with weights as e4m3
+ * codes times fp32 row scales:
+ *   score[t] = |s_gate[t]| sum_j |gate[t][j]| sqrt(h_in[j])
+ *            + |s_up[t]|   sum_j |up[t][j]|   sqrt(h_in[j])
+ *            + sqrt(h_mid[t]) sum_i |s_down[i]| |down[i][t]|
+ * computed in fp32 in a fixed order (repeatable bit for bit).
+ *   gate, up   device, e4m3 [I][H] row-major, 16-byte aligned; either may be
+ *              NULL (its term is left out). s_gate, s_up: device fp32 [I].
+ *   down       device, e4m3 [H][I] row-major, 16-byte aligned; s_down fp32 [H].
+ *   h_in       device fp32 [H], h_mid device fp32 [I]: the diagonals of the
+ *              input Hessians of gate/up and of down (non-negative).
+ *   I, H       multiples of 16 in [16, 2^20].
+ *   score      device fp32 [I] (caller-owned).
+ *   workspace  device, 256-byte aligned, at least spense_score_workspace_size(I, H)
+ *              bytes (no zeroing needed).
+ * Asynchronous on `stream`. The weights must hold no e4m3 NaN code (0x7F or
+ * 0xFF; spense_pack rejects them too): the score of a row or column with one
+ * is unspecified. Errors: ARG, SHAPE, ALIGN, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+SPENSE_API spense_status spense_score_glu(const uint8_t* gate, const float* s_gate, const uint8_t* up,
+                                          const float* s_up, int64_t I, int64_t H, const uint8_t* down,
+                                          const float* s_down, const float* h_in, const float* h_mid, float* score,
+                                          void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes spense_score_glu needs (0 for a bad shape). */
+SPENSE_API size_t spense_score_workspace_size(int64_t I, int64_t H);
+
+/*
+ * spense_select_dense — the dense set SpenseGPT+ keeps: the Kd indices with
+ * the largest scores, ties to the lower index, written in ascending order
+ * (ready for spense_pack's dense_idx after a copy to the host).
+ *   score      device fp32 [I], non-negative (as spense_score_glu writes).
+ *   I          1 .. 2^20;  Kd  0 .. I.
+ *   dense_idx  device int32 [Kd] (caller-owned).
+ * Asynchronous on `stream`. Errors: ARG, SHAPE, ALIGN, UNSUPPORTED, CUDA.
+ */
+SPENSE_API spense_status spense_select_dense(const float* score, int64_t I, int64_t Kd, int32_t* dense_idx,
+                                             void* stream);
+
+/*
  * spense_gemm_host — the same GEMM on HOST buffers: copies X [M][K] and
  * x_scale [M] from host memory into the workspace, runs spense_gemm, copies Y
  * [M][N] back to host memory and synchronizes `stream` before returning.

@@ -151,3 +151,23 @@ def test_quantize_without_a_device_reports_unsupported(L):
     if has_gpu:
         pytest.skip("a GPU is present")
     assert _quant_raw(L) == 11
+
+
+def test_score_and_select_reject_bad_arguments(L):
+    v = lambda a: ctypes.c_void_p(a) if a else None
+    def score(gate=0x1000, s_gate=0x2000, I=64, H=32, down=0x3000, s_down=0x4000, h_in=0x5000, h_mid=0x6000,
+              out=0x7000, ws=0x8000, ws_bytes=1 << 20):
+        return L.spense_score_glu(v(gate), v(s_gate), None, None, I, H, v(down), v(s_down), v(h_in), v(h_mid),
+                                  v(out), v(ws), ws_bytes, None)
+    assert score(down=0) == 1
+    assert score(s_gate=0) == 1                  # gate without its scales
+    assert score(I=60) == 2 and score(H=8) == 2
+    assert score(gate=0x1008) == 3 and score(h_in=0x5002) == 3
+    assert score(ws=0) == 7 and score(ws_bytes=16) == 7
+    assert score(ws=0x8010) == 3
+    assert L.spense_score_workspace_size(64, 32) >= 32 * 64 * 4
+    assert L.spense_score_workspace_size(60, 32) == 0
+    assert L.spense_select_dense(v(0x1000), 0, 0, v(0x2000), None) == 2
+    assert L.spense_select_dense(v(0x1000), 10, 11, v(0x2000), None) == 2
+    assert L.spense_select_dense(None, 10, 3, v(0x2000), None) == 1
+    assert L.spense_select_dense(v(0x1002), 10, 3, v(0x2000), None) == 3
