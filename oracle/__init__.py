@@ -221,6 +221,32 @@ def select_top(score, Kd):
     return out
 
 
+def output_split_keep(W, dense_rows):
+    """Keep mask [N, K] of an output-split weight (Technical Summary §2A:
+    output-split splits the output tensor, a sparse GEMM for one part and a
+    dense GEMM for the other): the rows in `dense_rows` keep every entry, every
+    other row is 2:4 over all K columns (its top two per group of four, as
+    `pack` with Kd = 0 selects them). Y = gemm(X, s_x, W, s_w, keep=...)."""
+    W = _u8(W)
+    N, K = W.shape
+    dense = np.zeros(N, bool)
+    dense[np.asarray(dense_rows, dtype=np.int64)] = True
+    keep = np.ones((N, K), np.uint8)
+    sparse_rows = np.flatnonzero(~dense)
+    if sparse_rows.size:
+        keep[sparse_rows] = pack(W[sparse_rows], Kd=0)["keep"]
+    return keep
+
+
+def glu_order(I, dense_idx):
+    """The order of the intermediate indices of a GLU MLP after its dense
+    indices are permuted into one contiguous block at the end (Technical
+    Summary §2B): the other indices ascending, then `dense_idx` ascending."""
+    d = np.asarray(dense_idx, dtype=np.int64)
+    rest = np.setdiff1d(np.arange(I, dtype=np.int64), d)
+    return np.concatenate([rest, np.sort(d)])
+
+
 def within_tolerance(y, yref, bound, rel=4e-3, absb=1e-5):
     """The acceptance rule |y - y_ref| <= 4e-3 |y_ref| + 1e-5 sum_k |w_k x_k|."""
     y = np.asarray(y, dtype=np.float64)
