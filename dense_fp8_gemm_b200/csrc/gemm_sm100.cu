@@ -117,34 +117,6 @@ __device__ __forceinline__ int block_owner(const GemmParams& p, int b) {
   return lo;
 }
 
-// The units (tile, block range) of one CTA's block range, in processing order:
-// a partial last unit is moved to the front, so both shared tiles come first.
-struct Units {
-  int nblk, t_first, j_first, t_last, j_last_end, count;
-  bool move_last;
-  __device__ Units(int b0, int b1, int nblk_) : nblk(nblk_) {
-    if (b1 <= b0) {
-      count = 0;
-      t_first = j_first = t_last = j_last_end = 0;
-      move_last = false;
-      return;
-    }
-    t_first = b0 / nblk;
-    j_first = b0 - t_first * nblk;
-    t_last = (b1 - 1) / nblk;
-    j_last_end = b1 - t_last * nblk;
-    count = t_last - t_first + 1;
-    move_last = count >= 2 && j_last_end < nblk;
-  }
-  // Unit at processing position u: tile t, blocks [j0, j1).
-  __device__ void get(int u, int& t, int& j0, int& j1) const {
-    const int k = move_last ? (u == 0 ? count - 1 : u - 1) : u;
-    t = t_first + k;
-    j0 = (k == 0) ? j_first : 0;
-    j1 = (k == count - 1) ? j_last_end : nblk;
-  }
-};
-
 // Group member holding global row tile n_tile.
 __device__ __forceinline__ int member_of(const GemmParams& p, int n_tile) {
   int i = 0;
@@ -153,6 +125,61 @@ __device__ __forceinline__ int member_of(const GemmParams& p, int n_tile) {
     if (k < p.n_members && p.mem[k].tile_begin <= n_tile) i = k;
   return i;
 }
+
+// First linear block of tile t (and, through nb, its number of blocks): a
+// member's tiles all have its layout and lie end to end from block_begin.
+__device__ __forceinline__ int tile_block0(const GemmParams& p, int t, int* nb) {
+  const GemmMember& mb = p.mem[member_of(p, t / p.m_tiles)];
+  if (nb != nullptr) *nb = mb.nblk;
+  return mb.block_begin + (t - mb.tile_begin * p.m_tiles) * mb.nblk;
+}
+
+// Tile t and block j within it of linear block b.
+__device__ __forceinline__ void block_tile(const GemmParams& p, int b, int& t, int& j) {
+  int i = 0;
+#pragma unroll
+  for (int k = 1; k < kMaxGroup; ++k)
+    if (k < p.n_members && p.mem[k].block_begin <= b) i = k;
+  const GemmMember& mb = p.mem[i];
+  const int local = b - mb.block_begin;
+  const int tl = local / mb.nblk;
+  t = mb.tile_begin * p.m_tiles + tl;
+  j = local - tl * mb.nblk;
+}
+
+// The units (tile, block range) of one CTA's block range, in processing order:
+// a partial last unit is moved to the front, so both shared tiles come first.
+struct Units {
+  const GemmParams* p;
+  int t_first, j_first, t_last, j_last_end, count;
+  bool move_last;
+  __device__ Units(const GemmParams& pp, int b0, int b1) : p(&pp) {
+    if (b1 <= b0) {
+      count = 0;
+      t_first = j_first = t_last = j_last_end = 0;
+      move_last = false;
+      return;
+    }
+    block_tile(pp, b0, t_first, j_first);
+    int jl;
+    block_tile(pp, b1 - 1, t_last, jl);
+    j_last_end = jl + 1;
+    count = t_last - t_first + 1;
+    move_last = count >= 2 && j_last_end < nblk_of(t_last);
+  }
+  __device__ int nblk_of(int t) const {
+    int nb;
+    tile_block0(*p, t, &nb);
+    return nb;
+  }
+  // Unit at processing position u: tile t, blocks [j0, j1).
+  __device__ void get(int u, int& t, int& j0, int& j1) const {
+    const int k = move_last ? (u == 0 ? count - 1 : u - 1) : u;
+    t = t_first + k;
+    j0 = (k == 0) ? j_first : 0;
+    j1 = (k == count - 1) ? j_last_end : nblk_of(t);
+  }
+};
 
 // Walks the blocks of a CTA in processing order without integer division on
 // the per-block path.
@@ -212,7 +239,6 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   // this grid's CTAs exit and wait (griddepcontrol.wait) before reading
   // anything this grid writes.
   ptx::griddep_launch_dependents();
-  const int nblk = p.nsb + p.ndb;
   const int b0 = p.cta_start[g];
   const int b1 = p.cta_start[g + 1];
 
@@ -244,7 +270,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       // chunks up to the valid tokens) as one bulk copy per peer. This precedes
       // its arrival on the cluster barrier, which every peer waits for
       // before its first store.
-      const int t = b0 / nblk;
+      int t, j_unused;
+      block_tile(p, b0, t, j_unused);
       const int m_valid = min(p.npad, p.M - (t % p.m_tiles) * kMaxTokenTile);
       const uint32_t bytes = static_cast<uint32_t>((p.cluster - 1) * ((m_valid + 15) >> 4)) * kTileRows * 64u;
       ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->peer_done), bytes);
@@ -271,7 +298,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     return bars->tmem_base;
   };
   volatile int* abort_flag = &bars->abort_flag;
-  const Units units(b0, b1, nblk);
+  const Units units(p, b0, b1);
   const uint32_t smem_base = ptx::smem_addr(smem);
 
   if (warp == 0 || warp == 6) {
@@ -317,15 +344,15 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         const uint32_t a_s = smem_base + s * p.stage_bytes;
         const uint32_t full = ptx::smem_addr(&bars->full[s]);
         const uint32_t piece = kBlockBytes / static_cast<uint32_t>(p.bulk_split);
-        if (c.j < p.nsb) {
-          const size_t blk = static_cast<size_t>(c.local_tile) * p.nsb + c.j;
+        if (c.j < mb.nsb) {
+          const size_t blk = static_cast<size_t>(c.local_tile) * mb.nsb + c.j;
           ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * xbytes);
           for (int q = 0; q < p.bulk_split; ++q)
             ptx::bulk_g2s(a_s + q * piece, mb.vs_t + blk * kBlockBytes + q * piece, piece, full, pol_w);
           ptx::bulk_g2s(a_s + kBlockBytes + p.b_bytes, mb.e_t + blk * kMetaBlockBytes, kMetaBlockBytes,
                         full, pol_w);
         } else {
-          const size_t blk = static_cast<size_t>(c.local_tile) * p.ndb + (c.j - p.nsb);
+          const size_t blk = static_cast<size_t>(c.local_tile) * mb.ndb + (c.j - mb.nsb);
           ptx::mbar_arrive_expect_tx(full, kBlockBytes + xbytes);
           for (int q = 0; q < p.bulk_split; ++q)
             ptx::bulk_g2s(a_s + q * piece, mb.wd_t + blk * kBlockBytes + q * piece, piece, full, pol_w);
@@ -335,11 +362,12 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         const int y0 = c.m_tile * kMaxTokenTile;
         const uint32_t b_s = smem_base + s * p.stage_bytes + kBlockBytes;
         const uint32_t full = ptx::smem_addr(&bars->full[s]);
-        if (c.j < p.nsb) {
+        const GemmMember& mb = p.mem[c.member];
+        if (c.j < mb.nsb) {
           ptx::tma_load_2d(b_s, &tmap_x, c.j * kSparseBlockCols, y0, full, pol_x);
           ptx::tma_load_2d(b_s + box, &tmap_x, c.j * kSparseBlockCols + 128, y0, full, pol_x);
         } else {
-          ptx::tma_load_2d(b_s, &tmap_x, p.Ks + (c.j - p.nsb) * kDenseBlockCols, y0, full, pol_x);
+          ptx::tma_load_2d(b_s, &tmap_x, mb.Ks + (c.j - mb.nsb) * kDenseBlockCols, y0, full, pol_x);
         }
       };
       BlockWalker cw(units, p);
@@ -354,12 +382,12 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         for (int i = pre; i < last; ++i, cp.advance(p)) {
           if (i % np != me) continue;
           const GemmMember& mb = p.mem[cp.member];
-          if (cp.j < p.nsb) {
-            const size_t blk = static_cast<size_t>(cp.local_tile) * p.nsb + cp.j;
+          if (cp.j < mb.nsb) {
+            const size_t blk = static_cast<size_t>(cp.local_tile) * mb.nsb + cp.j;
             ptx::prefetch_l2_bulk(mb.vs_t + blk * kBlockBytes, kBlockBytes);
             ptx::prefetch_l2_bulk(mb.e_t + blk * kMetaBlockBytes, kMetaBlockBytes);
           } else {
-            const size_t blk = static_cast<size_t>(cp.local_tile) * p.ndb + (cp.j - p.nsb);
+            const size_t blk = static_cast<size_t>(cp.local_tile) * mb.ndb + (cp.j - mb.nsb);
             ptx::prefetch_l2_bulk(mb.wd_t + blk * kBlockBytes, kBlockBytes);
           }
         }
@@ -402,6 +430,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * static_cast<uint32_t>(p.npad);
+        const int nsb_u = p.mem[member_of(p, t / p.m_tiles)].nsb;  // 2:4 blocks of this tile
         for (int j = j0; j < j1; ++j, ring.advance()) {
           if (!wait_bar(ptx::smem_addr(&bars->full[ring.s]), ring.ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
                         abort_flag)) {
@@ -412,7 +441,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
           const uint32_t a_s = smem_base + ring.s * p.stage_bytes;
           const uint32_t b_s = a_s + kBlockBytes;
           const uint32_t e_s = b_s + p.b_bytes;
-          if (j < p.nsb) {
+          if (j < nsb_u) {
             const uint32_t e_tmem = tmem_base + e_col0 + ebuf * 8u;
             ptx::tmem_cp_128x128b(e_tmem, ptx::desc_rows16(e_s));
             ptx::tmem_cp_128x128b(e_tmem + 4u, ptx::desc_rows16(e_s + 2048u));
@@ -477,9 +506,11 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       const int n = (n_tile - mb.tile_begin) * kTileRows + row;
       const bool row_ok = n < mb.N;
       const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
-      const int g_lo = block_owner(p, t * nblk);
-      const int g_hi = block_owner(p, t * nblk + nblk - 1);
-      const int lo_slot = (p.cta_start[g_lo] >= t * nblk) ? 0 : 1;
+      int nb_t;
+      const int tb = tile_block0(p, t, &nb_t);
+      const int g_lo = block_owner(p, tb);
+      const int g_hi = block_owner(p, tb + nb_t - 1);
+      const int lo_slot = (p.cta_start[g_lo] >= tb) ? 0 : 1;
       const float* lo_part =
           p.partials + (static_cast<size_t>(g_lo) * 2 + lo_slot) * slot_elems + static_cast<size_t>(row) * p.npad;
       const float* next_part =
@@ -526,7 +557,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             for (int i = 0; i < 4; ++i) {
               const int m = c0 + 4 * q + i;
               if (q < nq && m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] =
+                mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] =
                     to_bf16_bits(r4[i] * sw * (m0 == staged_m0 ? bars->sx[m] : __ldg(p.s_x + m0 + m)));
             }
           }
@@ -606,7 +637,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
           // Y tile staged as [16 tokens][128 rows] bf16 in the first ring stage
           // (idle: every copy has landed and every MMA has completed), then
           // written with 16-byte stores when the tile's rows are all in range.
-          const bool vec = (n_base + kTileRows <= mb.N) && (mb.N % 8 == 0);
+          const bool vec = (n_base + kTileRows <= mb.N) && (mb.ldy % 8 == 0);
           uint16_t* ystage = reinterpret_cast<uint16_t*>(smem);
           for (int c = 0; c < nchunk; ++c) {
             const int c0 = c * 16;
@@ -638,7 +669,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
                 const int idx = et + 128 * h;  // 16-byte piece: token idx / 16, rows 8 * (idx % 16) ..
                 const int m = c0 + (idx >> 4);
                 if (m < m_valid)
-                  ptx::st_global_v4(mb.y + static_cast<size_t>(m0 + m) * mb.N + n_base + 8 * (idx & 15),
+                  ptx::st_global_v4(mb.y + static_cast<size_t>(m0 + m) * mb.ldy + n_base + 8 * (idx & 15),
                                     reinterpret_cast<const uint4*>(ystage)[idx]);
               }
             } else if (row_ok) {
@@ -646,7 +677,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
               for (int i = 0; i < 16; ++i) {
                 const int m = c0 + i;
                 if (m < m_valid)
-                  mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(a[i] * sw * bars->sx[m]);
+                  mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] = to_bf16_bits(a[i] * sw * bars->sx[m]);
               }
             }
           }
@@ -665,7 +696,9 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       const int m_valid = min(p.npad, p.M - m0);
       const int n = (n_tile - mb.tile_begin) * kTileRows + row;
       const bool row_ok = n < mb.N;
-      const bool whole = (j0 == 0 && j1 == nblk);
+      int nb_t;
+      const int tb = tile_block0(p, t, &nb_t);
+      const bool whole = (j0 == 0 && j1 == nb_t);
       const float sw = (row_ok && whole) ? __ldg(mb.s_w + n) : 0.0f;
       if (whole) stage_sx(m0);
       const bool got = wait_bar(ptx::smem_addr(&bars->acc_full[acc]), aph, p.status,
@@ -678,7 +711,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       // CTA's first block, slot 1 for the tile holding its last block.
       float* part = nullptr;
       if (!whole) {
-        const int slot = (b0 >= t * nblk) ? 0 : 1;
+        const int slot = (b0 >= tb) ? 0 : 1;
         part = p.partials + (static_cast<size_t>(g) * 2 + slot) * slot_elems + static_cast<size_t>(row) * p.npad;
       }
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
@@ -691,7 +724,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             for (int i = 0; i < 16; ++i) {
               const int m = c0 + i;
               if (m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.N + n] = to_bf16_bits(__uint_as_float(v[i]) * sw * bars->sx[m]);
+                mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] = to_bf16_bits(__uint_as_float(v[i]) * sw * bars->sx[m]);
             }
           }
         } else {
@@ -710,8 +743,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         // stores before thread 0's release-acquire ticket at GPU scope.
         ptx::named_bar_sync(1, 128);
         if (et == 0) {
-          const int g_lo = block_owner(p, t * nblk);
-          const int g_hi = block_owner(p, t * nblk + nblk - 1);
+          const int g_lo = block_owner(p, tb);
+          const int g_hi = block_owner(p, tb + nb_t - 1);
           const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
           bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
         }
@@ -724,7 +757,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       if (u + 1 < units.count) {
         int t2, a2, b2;
         units.get(u + 1, t2, a2, b2);
-        next_whole = (a2 == 0 && b2 == nblk);
+        next_whole = (a2 == 0 && b2 == units.nblk_of(t2));
       }
       if (next_whole) {
         for (int i = 0; i < npending; ++i) finish_tile(pending[i]);

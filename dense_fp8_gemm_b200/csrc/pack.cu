@@ -162,6 +162,22 @@ __global__ void __launch_bounds__(256) pack_dense_kernel(
 }
 
 // X'[m][j] = X[m][perm[j]]; one thread per 4 output bytes.
+// dst row r = src row rows[r] (K bytes each, K % 16 == 0), and the same for
+// one float per row when scales are given.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restrict__ src, int64_t K,
+                                                          const int32_t* __restrict__ rows, int64_t N,
+                                                          uint8_t* __restrict__ dst, const float* __restrict__ ssrc,
+                                                          float* __restrict__ sdst) {
+  const int64_t q = K / 16;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < N * q;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = t / q, c = t - r * q;
+    const int64_t sr = rows[r];
+    reinterpret_cast<uint4*>(dst + r * K)[c] = reinterpret_cast<const uint4*>(src + sr * K)[c];
+    if (c == 0 && ssrc != nullptr) sdst[r] = ssrc[sr];
+  }
+}
+
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ X,
                                                      const int32_t* __restrict__ perm, int64_t M,
                                                      int64_t K, uint8_t* __restrict__ Xg) {
@@ -214,6 +230,14 @@ cudaError_t launch_pack(const uint8_t* W, const uint8_t* mask, const int32_t* pe
     if (st != cudaSuccess) return st;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_gather_rows(const uint8_t* src, int64_t K, const int32_t* rows, int64_t N, uint8_t* dst,
+                               const float* ssrc, float* sdst, cudaStream_t stream) {
+  const int64_t threads = N * (K / 16);
+  const unsigned int grid = static_cast<unsigned int>(std::min<int64_t>(blocks_for(threads), 4096));
+  gather_rows_kernel<<<grid, 256, 0, stream>>>(src, K, rows, N, dst, ssrc, sdst);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gather(const uint8_t* X, const int32_t* perm, int64_t M, int64_t K, uint8_t* Xg,

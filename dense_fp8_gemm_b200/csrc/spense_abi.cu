@@ -174,36 +174,50 @@ int bulk_split() {
   return v;
 }
 
-// Checks that `count` handles can share one launch (same device, K, Kd and
-// dense column set) and plans it for M tokens on a device with `sms` SMs.
+// Checks that `count` handles can share one launch and plans it for M tokens
+// on a device with `sms` SMs. Members share the device, K and the column order
+// of X: either none has a scattered dense set (their Kd may differ, e.g. the
+// 2:4 rows and the dense rows of an output-split weight), or all have the
+// same one.
 spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, int sms, GemmPlan* out) {
   if (hs == nullptr || count < 1 || count > kMaxGroup)
     return fail(SPENSE_ERR_ARG, "a launch takes 1 to %d packed weights, got %d", kMaxGroup, count);
   if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
   const spense_packed* h0 = hs[0];
   if (h0 == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
-  long long n_tiles = 0;
-  for (int i = 0; i < count; ++i) {
-    const spense_packed* h = hs[i];
-    if (h == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
-    if (h->device != h0->device || h->K != h0->K || h->Kd != h0->Kd || h->perm_host != h0->perm_host)
-      return fail(SPENSE_ERR_ARG,
-                  "packed weights sharing a launch need the same device, K, Kd and dense column set");
-    n_tiles += h->n_tiles;
-  }
   GemmPlan pl{};
   pl.npad = M > kMaxTokenTile ? kMaxTokenTile : static_cast<int>(round_up(static_cast<size_t>(M), 16));
   pl.box_rows = static_cast<int>(M > kMaxTokenTile ? kMaxTokenTile : M);
   pl.m_tiles = static_cast<int>((M + kMaxTokenTile - 1) / kMaxTokenTile);
-  pl.nsb = h0->nsb;
-  pl.ndb = h0->ndb;
-  const long long nblk = pl.nsb + pl.ndb;
-  if (n_tiles * pl.m_tiles * nblk >= (1ll << 31))
-    return fail(SPENSE_ERR_SHAPE, "too many blocks for one launch (%lld)", n_tiles * pl.m_tiles * nblk);
+  pl.count = count;
+  long long n_tiles = 0, blocks = 0, cost = 0;
+  pl.min_tile_cost = 1 << 30;
+  pl.any_sparse = false;
+  for (int i = 0; i < count; ++i) {
+    const spense_packed* h = hs[i];
+    if (h == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
+    if (h->device != h0->device || h->K != h0->K || h->perm_host != h0->perm_host)
+      return fail(SPENSE_ERR_ARG,
+                  "packed weights sharing a launch need the same device, K and column order of X (the same "
+                  "scattered dense set, or none)");
+    pl.mem_tiles[i] = h->n_tiles;
+    pl.mem_nsb[i] = h->nsb;
+    pl.mem_ndb[i] = h->ndb;
+    pl.mem_cost[i] = kCostSparse * h->nsb + kCostDense * h->ndb;
+    pl.mem_block_begin[i] = static_cast<int>(std::min<long long>(blocks, 1ll << 31));
+    pl.mem_cost_begin[i] = cost;
+    const long long tiles_i = static_cast<long long>(h->n_tiles) * pl.m_tiles;
+    blocks += tiles_i * (h->nsb + h->ndb);
+    cost += tiles_i * pl.mem_cost[i];
+    n_tiles += h->n_tiles;
+    pl.min_tile_cost = std::min(pl.min_tile_cost, pl.mem_cost[i]);
+    pl.any_sparse = pl.any_sparse || h->nsb > 0;
+  }
+  pl.mem_cost_begin[count] = cost;
+  if (blocks >= (1ll << 31)) return fail(SPENSE_ERR_SHAPE, "too many blocks for one launch (%lld)", blocks);
   pl.n_tiles = static_cast<int>(n_tiles);
   pl.tiles = pl.n_tiles * pl.m_tiles;
-  pl.tile_cost = kCostSparse * pl.nsb + kCostDense * pl.ndb;
-  pl.total_cost = static_cast<long long>(pl.tiles) * pl.tile_cost;
+  pl.total_cost = cost;
   // Each CTA gets at least min_cta_weight() units of streamed bytes (never less
   // than one maximal block, so no CTA owns an empty range): small matrices are
   // split across fewer CTAs, which keeps the number of partials per tile low.
@@ -212,8 +226,8 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // in half the shared and tensor memory; otherwise one.
   pl.bulk_split = bulk_split();
   pl.producers = producers();
-  pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.nsb > 0 ? 256u : 128u);
-  pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.nsb > 0 ? kMetaBlockBytes : 0);
+  pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.any_sparse ? 256u : 128u);
+  pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.any_sparse ? kMetaBlockBytes : 0);
   const uint32_t reserve = 1024 + kBarrierBytes;  // alignment slack + barrier area
   const int cps_first =
       ctas_per_sm_knob() != 0 ? ctas_per_sm_knob() : ((pl.tiles > 2 * sms || pl.npad > 32) ? 1 : 2);
@@ -233,10 +247,27 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   }
   const long long slots =
       std::min<long long>(static_cast<long long>(sms) * std::min(pl.ctas_per_sm, grid_per_sm()), kMaxGrid);
-  // First block of a tile whose start weight is >= c (c within one tile).
-  auto block_at = [&](long long c) {
-    const long long sp = static_cast<long long>(kCostSparse) * pl.nsb;
-    return c <= sp ? (c + kCostSparse - 1) / kCostSparse : pl.nsb + (c - sp + kCostDense - 1) / kCostDense;
+  // First block of a tile of member i whose start weight is >= c (c within one tile).
+  auto block_at = [&](int i, long long c) {
+    const long long sp = static_cast<long long>(kCostSparse) * pl.mem_nsb[i];
+    return c <= sp ? (c + kCostSparse - 1) / kCostSparse : pl.mem_nsb[i] + (c - sp + kCostDense - 1) / kCostDense;
+  };
+  // Member of global tile t (tiles of a member are consecutive).
+  auto member_of_tile = [&](long long t) {
+    int i = 0;
+    long long acc = 0;
+    for (; i < count - 1; ++i) {
+      acc += static_cast<long long>(pl.mem_tiles[i]) * pl.m_tiles;
+      if (t < acc) break;
+    }
+    return i;
+  };
+  // First linear block of global tile t.
+  auto tile_block0 = [&](long long t) {
+    const int i = member_of_tile(t);
+    long long first_tile = 0;
+    for (int k = 0; k < i; ++k) first_tile += static_cast<long long>(pl.mem_tiles[k]) * pl.m_tiles;
+    return pl.mem_block_begin[i] + (t - first_tile) * (pl.mem_nsb[i] + pl.mem_ndb[i]);
   };
   // Few tiles (at most half the CTA slots): the CTAs of a cluster of S split
   // each tile's K range by weight and reduce in shared memory; otherwise
@@ -250,7 +281,7 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     // them, unless the GEMM is so small that fixed costs dominate anyway.
     for (int S = 8; S >= 2; S >>= 1) {
       if (mode > 1 && S != mode) continue;
-      if (pl.tiles * S > slots || S > pl.tile_cost / kCostSparse) continue;
+      if (pl.tiles * S > slots || S > pl.min_tile_cost / kCostSparse) continue;
       const bool fills = pl.tiles * S * 2 >= slots;
       const bool small = pl.total_cost < 40LL * slots;
       if (mode > 1 || fills || small) {
@@ -277,7 +308,13 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     pl.grid = pl.tiles * pl.cluster;
     for (int g = 0; g <= pl.grid; ++g) {
       const long long t = g / pl.cluster, r = g % pl.cluster;
-      pl.cta_start[g] = static_cast<int>(t * nblk + block_at((r * pl.tile_cost + pl.cluster - 1) / pl.cluster));
+      if (t >= pl.tiles) {
+        pl.cta_start[g] = static_cast<int>(blocks);
+        continue;
+      }
+      const int i = member_of_tile(t);
+      pl.cta_start[g] = static_cast<int>(tile_block0(t) + block_at(i, (r * pl.mem_cost[i] + pl.cluster - 1) /
+                                                                             pl.cluster));
     }
   } else {
     grid = std::max<long long>(1, std::min<long long>(grid, slots));
@@ -285,8 +322,16 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     // CTA g takes the blocks whose start weight falls in [g T / G, (g+1) T / G).
     for (int g = 0; g <= pl.grid; ++g) {
       const long long c = (static_cast<long long>(g) * pl.total_cost + pl.grid - 1) / pl.grid;
-      const long long t = c / pl.tile_cost;
-      pl.cta_start[g] = static_cast<int>(t * nblk + block_at(c - t * pl.tile_cost));
+      if (c >= pl.total_cost) {
+        pl.cta_start[g] = static_cast<int>(blocks);
+        continue;
+      }
+      int i = 0;
+      while (i + 1 < count && c >= pl.mem_cost_begin[i + 1]) ++i;
+      const long long ci = c - pl.mem_cost_begin[i];
+      const long long tl = ci / pl.mem_cost[i];  // tile within member i
+      pl.cta_start[g] = static_cast<int>(pl.mem_block_begin[i] + tl * (pl.mem_nsb[i] + pl.mem_ndb[i]) +
+                                         block_at(i, ci - tl * pl.mem_cost[i]));
     }
   }
   pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes + pl.recv_bytes;
@@ -334,7 +379,7 @@ spense_status check_gemm_args(const spense_packed* const* hs, int count, int64_t
 // Enqueue one launch over `count` packed weights sharing X (arguments validated).
 spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t* X, const float* x_scale,
                        int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream,
-                       bool x_packed_order = false) {
+                       bool x_packed_order = false, const int64_t* ldy = nullptr) {
   const spense_packed* h0 = hs[0];
   const uint8_t* xsrc = X;
   if (h0->perm != nullptr && !x_packed_order) {
@@ -366,6 +411,12 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
     m.y = Ys[i];
     m.N = static_cast<int>(hs[i]->N);
     m.tile_begin = tile_begin;
+    m.nsb = pl.mem_nsb[i];
+    m.ndb = pl.mem_ndb[i];
+    m.nblk = m.nsb + m.ndb;
+    m.Ks = static_cast<int>(hs[i]->Ks);
+    m.block_begin = pl.mem_block_begin[i];
+    m.ldy = static_cast<int>(ldy != nullptr ? ldy[i] : hs[i]->N);
     tile_begin += hs[i]->n_tiles;
   }
   p.n_members = count;
@@ -374,12 +425,8 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
   p.counters = reinterpret_cast<unsigned int*>(ws + pl.ws.counters_off);
   p.status = reinterpret_cast<unsigned int*>(ws);
   p.M = static_cast<int>(M);
-  p.Ks = static_cast<int>(h0->Ks);
-  p.Kd = static_cast<int>(h0->Kd);
   p.n_tiles = pl.n_tiles;
   p.m_tiles = pl.m_tiles;
-  p.nsb = pl.nsb;
-  p.ndb = pl.ndb;
   p.npad = pl.npad;
   p.box_rows = pl.box_rows;
   p.grid = pl.grid;
@@ -432,6 +479,51 @@ extern "C" {
 const char* spense_last_error(void) { return g_last_error.c_str(); }
 
 const char* spense_version(void) { return "0.1.0"; }
+
+spense_status spense_pack_rows(const uint8_t* W, const float* w_scale, int64_t N_src, int64_t K,
+                               const int32_t* rows, int64_t N, const uint8_t* mask, const int32_t* dense_idx,
+                               int64_t Kd, uint32_t flags, void* stream_v, spense_packed** out) {
+  if (out == nullptr) return fail(SPENSE_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  if (W == nullptr || w_scale == nullptr || rows == nullptr) return fail(SPENSE_ERR_ARG, "W, w_scale or rows is NULL");
+  if (N_src < 1 || N_src > (1 << 20) || N < 1 || N > (1 << 20))
+    return fail(SPENSE_ERR_SHAPE, "N_src = %lld and N = %lld must be in [1, 2^20]", (long long)N_src, (long long)N);
+  if (K < 16 || K > (1 << 20) || K % 16 != 0)
+    return fail(SPENSE_ERR_SHAPE, "K = %lld must be a multiple of 16 in [16, 2^20]", (long long)K);
+  if (!aligned(W, 16) || (mask != nullptr && !aligned(mask, 16)) || !aligned(w_scale, 4))
+    return fail(SPENSE_ERR_ALIGN, "W and mask must be 16-byte aligned, w_scale 4-byte aligned");
+  for (int64_t r = 0; r < N; ++r)
+    if (rows[r] < 0 || rows[r] >= N_src)
+      return fail(SPENSE_ERR_ARG, "rows[%lld] = %d outside [0, %lld)", (long long)r, rows[r], (long long)N_src);
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  // Gather the rows into temporaries, pack those, free them (pack synchronizes).
+  uint8_t* wt = nullptr;
+  uint8_t* mt = nullptr;
+  float* st_ = nullptr;
+  int32_t* rd = nullptr;
+  const size_t bytes = static_cast<size_t>(N) * static_cast<size_t>(K);
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&wt), bytes);
+  if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&st_), static_cast<size_t>(N) * 4);
+  if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&rd), static_cast<size_t>(N) * 4);
+  if (e == cudaSuccess && mask != nullptr) e = cudaMalloc(reinterpret_cast<void**>(&mt), bytes);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(rd, rows, static_cast<size_t>(N) * 4, cudaMemcpyHostToDevice, stream);
+  if (e == cudaSuccess) e = launch_gather_rows(W, K, rd, N, wt, w_scale, st_, stream);
+  if (e == cudaSuccess && mask != nullptr) e = launch_gather_rows(mask, K, rd, N, mt, nullptr, nullptr, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // `rows` may be a host temporary
+  if (e != cudaSuccess) {
+    for (void* q : {static_cast<void*>(wt), static_cast<void*>(mt), static_cast<void*>(st_), static_cast<void*>(rd)})
+      if (q != nullptr) cudaFree(q);
+    return cuda_fail(e, "row gather");
+  }
+  st = spense_pack(wt, st_, N, K, mt, dense_idx, Kd, flags, stream_v, out);
+  for (void* q : {static_cast<void*>(wt), static_cast<void*>(mt), static_cast<void*>(st_), static_cast<void*>(rd)})
+    if (q != nullptr) cudaFree(q);
+  return st;
+}
 
 spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int64_t K,
                           const uint8_t* mask, const int32_t* dense_idx, int64_t Kd, uint32_t flags,
@@ -565,12 +657,12 @@ size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M) {
 spense_status spense_gemm_grouped(const spense_packed* const* Wps, int count, const uint8_t* X,
                                   const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
                                   size_t workspace_bytes, void* stream_v) {
-  return spense_gemm_grouped_ex(Wps, count, X, x_scale, M, Ys, workspace, workspace_bytes, 0u, stream_v);
+  return spense_gemm_grouped_ex(Wps, count, X, x_scale, M, Ys, nullptr, workspace, workspace_bytes, 0u, stream_v);
 }
 
 spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count, const uint8_t* X,
-                                     const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
-                                     size_t workspace_bytes, unsigned int flags, void* stream_v) {
+                                     const float* x_scale, int64_t M, uint16_t* const* Ys, const int64_t* ldy,
+                                     void* workspace, size_t workspace_bytes, unsigned int flags, void* stream_v) {
   if ((flags & ~static_cast<unsigned int>(SPENSE_GEMM_X_PACKED_ORDER)) != 0u)
     return fail(SPENSE_ERR_ARG, "unknown flags %#x", flags);
   if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
@@ -581,6 +673,9 @@ spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count,
     for (int i = 0; i < count; ++i) {
       if (Ys[i] == nullptr) return fail(SPENSE_ERR_ARG, "Y[%d] is NULL", i);
       if (!aligned(Ys[i], 16)) return fail(SPENSE_ERR_ALIGN, "Y[%d] must be 16-byte aligned", i);
+      if (ldy != nullptr && Wps != nullptr && Wps[i] != nullptr &&
+          (ldy[i] < Wps[i]->N || ldy[i] > (1ll << 30)))
+        return fail(SPENSE_ERR_SHAPE, "ldy[%d] = %lld is smaller than N or too large", i, (long long)ldy[i]);
     }
   }
   DeviceInfo info;
@@ -593,7 +688,7 @@ spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count,
     return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
                 pl.ws.total_device);
   st = run_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
-                static_cast<cudaStream_t>(stream_v), (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u);
+                static_cast<cudaStream_t>(stream_v), (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u, ldy);
   return st == SPENSE_OK ? ok() : st;
 }
 

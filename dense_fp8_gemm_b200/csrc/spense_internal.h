@@ -42,8 +42,14 @@ struct GemmPlan {
   int m_tiles;
   int n_tiles;     // row tiles over all group members
   int tiles;       // n_tiles * m_tiles
-  int nsb, ndb;    // sparse / dense blocks per tile
-  int tile_cost;   // kCostSparse * nsb + kCostDense * ndb
+  int count;                                // weight matrices in the launch
+  int mem_tiles[kMaxGroup];                 // row tiles of member i
+  int mem_nsb[kMaxGroup], mem_ndb[kMaxGroup];  // 2:4 / dense blocks per tile of member i
+  int mem_cost[kMaxGroup];                  // kCostSparse * nsb + kCostDense * ndb
+  int mem_block_begin[kMaxGroup];           // first linear block of member i
+  long long mem_cost_begin[kMaxGroup + 1];  // streamed weight before member i's first tile
+  int min_tile_cost;
+  bool any_sparse;
   long long total_cost;
   int grid;        // CTAs
   int stages;
@@ -68,9 +74,14 @@ struct GemmMember {
   const uint8_t* e_t;
   const uint8_t* wd_t;
   const float* s_w;
-  uint16_t* y;
+  uint16_t* y;       // row m of the output at y + m * ldy
   int N;
-  int tile_begin;
+  int tile_begin;    // first global row tile
+  int nsb, ndb;      // 2:4 blocks and dense blocks per row tile
+  int nblk;          // nsb + ndb
+  int Ks;            // X column where the dense region starts
+  int block_begin;   // first linear block of the member's tiles
+  int ldy;           // output row stride in elements (>= N)
 };
 
 struct GemmParams {
@@ -80,8 +91,8 @@ struct GemmParams {
   float* partials;
   unsigned int* counters;
   unsigned int* status;
-  int M, Ks, Kd;
-  int n_tiles, m_tiles, nsb, ndb;
+  int M;
+  int n_tiles, m_tiles;
   int npad, box_rows, grid, stages, nacc;
   uint32_t stage_bytes, b_bytes;
   uint32_t tmem_cols;
@@ -101,6 +112,8 @@ cudaError_t launch_pack(const uint8_t* W, const uint8_t* mask, const int32_t* pe
                         cudaStream_t stream);
 cudaError_t launch_gather(const uint8_t* X, const int32_t* perm, int64_t M, int64_t K, uint8_t* Xg,
                           cudaStream_t stream);
+cudaError_t launch_gather_rows(const uint8_t* src, int64_t K, const int32_t* rows, int64_t N, uint8_t* dst,
+                               const float* ssrc, float* sdst, cudaStream_t stream);
 cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t smem_bytes,
                         cudaStream_t stream);
 uint32_t gemm_max_smem();

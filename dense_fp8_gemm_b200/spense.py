@@ -30,6 +30,7 @@ SYMBOLS = (
     "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
     "spense_gemm_grouped", "spense_gemm_grouped_workspace_size", "spense_gemm_grouped_ex",
     "spense_quantize", "spense_score_glu", "spense_score_workspace_size", "spense_select_dense",
+    "spense_pack_rows",
 )
 GEMM_X_PACKED_ORDER = 1
 MAX_GROUP = 4
@@ -78,8 +79,9 @@ def lib() -> ctypes.CDLL:
     L.spense_gemm_grouped.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ, P]
     L.spense_gemm_grouped_workspace_size.argtypes = [ctypes.POINTER(P), ctypes.c_int, I64]
     L.spense_gemm_grouped_workspace_size.restype = SZ
-    L.spense_gemm_grouped_ex.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ,
-                                         U32, P]
+    L.spense_gemm_grouped_ex.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, P,
+                                         SZ, U32, P]
+    L.spense_pack_rows.argtypes = [P, P, I64, I64, P, I64, P, P, I64, U32, P, ctypes.POINTER(P)]
     L.spense_quantize.argtypes = [P, I64, I64, P, P, P, P]
     L.spense_score_glu.argtypes = [P, P, P, P, I64, I64, P, P, P, P, P, P, SZ, P]
     L.spense_score_workspace_size.argtypes = [I64, I64]
@@ -187,8 +189,9 @@ class PackedWeight:
 
 
 def pack(W: torch.Tensor, w_scale: torch.Tensor, Kd: int | None = None, mask: torch.Tensor | None = None,
-         dense_idx=None, keep_canonical: bool = False, stream=None) -> PackedWeight:
-    """spense_pack. W: uint8 [N, K] (e4m3 bytes) on the GPU; w_scale fp32 [N];
+         dense_idx=None, keep_canonical: bool = False, stream=None, rows=None) -> PackedWeight:
+    """spense_pack, or spense_pack_rows when `rows` (host int32 row indices) is
+    given. W: uint8 [N, K] (e4m3 bytes) on the GPU; w_scale fp32 [N];
     dense_idx: host int32 index list (SpenseGPT+) or None (tail of Kd columns)."""
     N, K = W.shape
     idx = None
@@ -200,12 +203,20 @@ def pack(W: torch.Tensor, w_scale: torch.Tensor, Kd: int | None = None, mask: to
     if Kd is None:
         raise ValueError("Kd (or dense_idx) is required")
     out = ctypes.c_void_p()
-    code = lib().spense_pack(
-        _dev_ptr(W, torch.uint8, "W"), _dev_ptr(w_scale, torch.float32, "w_scale"), N, K,
-        _dev_ptr(mask, torch.uint8, "mask"),
-        None if idx is None else idx.ctypes.data_as(ctypes.c_void_p), Kd,
-        PACK_KEEP_CANONICAL if keep_canonical else 0, _stream(stream), ctypes.byref(out))
-    _check(code, "spense_pack")
+    flags = PACK_KEEP_CANONICAL if keep_canonical else 0
+    dptr = None if idx is None else idx.ctypes.data_as(ctypes.c_void_p)
+    if rows is None:
+        code = lib().spense_pack(
+            _dev_ptr(W, torch.uint8, "W"), _dev_ptr(w_scale, torch.float32, "w_scale"), N, K,
+            _dev_ptr(mask, torch.uint8, "mask"), dptr, Kd, flags, _stream(stream), ctypes.byref(out))
+        _check(code, "spense_pack")
+    else:
+        r = np.ascontiguousarray(np.asarray(rows), dtype=np.int32)
+        code = lib().spense_pack_rows(
+            _dev_ptr(W, torch.uint8, "W"), _dev_ptr(w_scale, torch.float32, "w_scale"), N, K,
+            r.ctypes.data_as(ctypes.c_void_p), r.shape[0], _dev_ptr(mask, torch.uint8, "mask"), dptr, Kd, flags,
+            _stream(stream), ctypes.byref(out))
+        _check(code, "spense_pack_rows")
     return PackedWeight(out)
 
 
@@ -275,25 +286,40 @@ def grouped_workspace_size(pws, M: int) -> int:
 
 
 def gemm_grouped(pws, X: torch.Tensor, x_scale: torch.Tensor, Ys=None, workspace: torch.Tensor | None = None,
-                 stream=None, flags: int = 0):
-    """spense_gemm_grouped (flags == 0) or spense_gemm_grouped_ex: one launch
-    over several packed weights sharing X (same K, Kd and dense column set).
-    flags = GEMM_X_PACKED_ORDER: X is already in the packed column order (from
-    quantize(..., order=pw)). Returns the list of outputs."""
+                 stream=None, flags: int = 0, ldy=None):
+    """spense_gemm_grouped (flags == 0, ldy None) or spense_gemm_grouped_ex:
+    one launch over several packed weights sharing X (same K and column order
+    of X). flags = GEMM_X_PACKED_ORDER: X is already in the packed column order
+    (from quantize(..., order=pw)). ldy: per-output row strides in elements,
+    with Ys given as flat device tensors (views into a wider output). Returns
+    the list of outputs."""
     M = X.shape[0]
     if Ys is None:
         Ys = [torch.empty((M, pw.N), dtype=torch.bfloat16, device=X.device) for pw in pws]
     if workspace is None:
         workspace = new_workspace(grouped_workspace_size(pws, M), X.device)
     yarr = (ctypes.c_void_p * len(pws))()
+    strided = any(not Y.is_contiguous() for Y in Ys)
+    if strided and ldy is None:
+        ldy = [Y.stride(0) for Y in Ys]  # column slices of a wider output
     for i, Y in enumerate(Ys):
-        yarr[i] = _dev_ptr(Y, torch.bfloat16, f"Y[{i}]").value
-    args = (_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"), _dev_ptr(x_scale, torch.float32, "x_scale"),
-            M, yarr, _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel())
-    if flags == 0:
-        _check(lib().spense_gemm_grouped(*args, _stream(stream)), "spense_gemm_grouped")
+        if Y.is_contiguous():
+            yarr[i] = _dev_ptr(Y, torch.bfloat16, f"Y[{i}]").value
+        else:
+            if not Y.is_cuda or Y.dtype != torch.bfloat16 or Y.stride(1) != 1:
+                raise ValueError(f"Y[{i}] must be a bfloat16 CUDA tensor with unit column stride")
+            yarr[i] = Y.data_ptr()
+    if flags == 0 and ldy is None:
+        _check(lib().spense_gemm_grouped(_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"),
+                                         _dev_ptr(x_scale, torch.float32, "x_scale"), M, yarr,
+                                         _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                         _stream(stream)), "spense_gemm_grouped")
     else:
-        _check(lib().spense_gemm_grouped_ex(*args, int(flags), _stream(stream)), "spense_gemm_grouped_ex")
+        larr = None if ldy is None else (ctypes.c_int64 * len(pws))(*[int(v) for v in ldy])
+        _check(lib().spense_gemm_grouped_ex(_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"),
+                                            _dev_ptr(x_scale, torch.float32, "x_scale"), M, yarr, larr,
+                                            _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                            int(flags), _stream(stream)), "spense_gemm_grouped_ex")
     return Ys
 
 

@@ -113,6 +113,23 @@ SPENSE_API spense_status spense_pack(const uint8_t* W, const float* w_scale, int
                           uint32_t flags, void* stream, spense_packed** out);
 
 /*
+ * spense_pack_rows — spense_pack of the rows W[rows[r]], r = 0 .. N-1, of a
+ * matrix W [N_src][K] (and the same rows of w_scale and of the mask). The
+ * rows are gathered on the device into a temporary before packing. Used for
+ * the output-split execution (Technical Summary §2.A: the output channels are
+ * split into a 2:4 part and a dense part) and to fold the SpenseGPT+
+ * permutation of the intermediate indices into the gate and up rows
+ * (Technical Summary §2.B: permuting the intermediate indices of a GLU MLP
+ * leaves its output unchanged).
+ *   rows   HOST int32 [N], each in [0, N_src) (repeats allowed).
+ * Other arguments and errors as spense_pack (ARG also for a bad row index).
+ */
+SPENSE_API spense_status spense_pack_rows(const uint8_t* W, const float* w_scale, int64_t N_src, int64_t K,
+                                          const int32_t* rows, int64_t N, const uint8_t* mask,
+                                          const int32_t* dense_idx, int64_t Kd, uint32_t flags, void* stream,
+                                          spense_packed** out);
+
+/*
  * spense_gemm — Y = X * Wm^T with scales (Technical Summary §2.A input-split,
  * both regions into one fp32 accumulator; §2.B the activations are gathered
  * into the packed column order when dense_idx was given).
@@ -169,13 +186,23 @@ enum {
 };
 
 /*
- * spense_gemm_grouped_ex — spense_gemm_grouped with flags (above); unknown
- * flag bits are an ARG error. With flags == 0 it is spense_gemm_grouped.
+ * spense_gemm_grouped_ex — spense_gemm_grouped with output strides and flags.
+ * Members need the same device, K and column order of X, but when none has a
+ * scattered dense set their Kd may differ: a weight packed with Kd = 0 (all
+ * 2:4) and one packed with Kd = K (all dense) can share a launch. That is the
+ * output-split execution of Technical Summary §2.A (the output channels split
+ * into a 2:4 part and a dense part): pack the two row sets with
+ * spense_pack_rows and point their outputs into one Y with ldy = N_total.
+ *   ldy    NULL: Ys[i] is [M][N_i] contiguous. Else host int64 [count]: row m
+ *          of output i starts at Ys[i] + m * ldy[i], N_i <= ldy[i] <= 2^30
+ *          (16-byte stores are used when ldy[i] % 8 == 0).
+ *   flags  0 or SPENSE_GEMM_X_PACKED_ORDER; unknown bits are an ARG error.
+ * With ldy == NULL and flags == 0 it is spense_gemm_grouped.
  */
 SPENSE_API spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count, const uint8_t* X,
                                                 const float* x_scale, int64_t M, uint16_t* const* Ys,
-                                                void* workspace, size_t workspace_bytes, unsigned int flags,
-                                                void* stream);
+                                                const int64_t* ldy, void* workspace, size_t workspace_bytes,
+                                                unsigned int flags, void* stream);
 
 /*
  * spense_quantize — per-token FP8 quantisation of bf16 activations, the step in

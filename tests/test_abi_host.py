@@ -137,7 +137,7 @@ def test_quantize_rejects_bad_arguments(L):
 def test_gemm_ex_rejects_unknown_flags(L):
     h = (ctypes.c_void_p * 1)(0x10)
     y = (ctypes.c_void_p * 1)(0x3000)
-    code = L.spense_gemm_grouped_ex(h, 1, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 1, y,
+    code = L.spense_gemm_grouped_ex(h, 1, ctypes.c_void_p(0x1000), ctypes.c_void_p(0x2000), 1, y, None,
                                     ctypes.c_void_p(0x4000), 1 << 20, 0x2, None)
     assert code == 1 and b"flags" in L.spense_last_error()
 
@@ -171,3 +171,17 @@ def test_score_and_select_reject_bad_arguments(L):
     assert L.spense_select_dense(v(0x1000), 10, 11, v(0x2000), None) == 2
     assert L.spense_select_dense(None, 10, 3, v(0x2000), None) == 1
     assert L.spense_select_dense(v(0x1002), 10, 3, v(0x2000), None) == 3
+
+
+def test_pack_rows_rejects_bad_arguments(L):
+    out = ctypes.c_void_p(0x1234)
+    rows = (ctypes.c_int32 * 3)(0, 5, 2)
+    v = lambda a: ctypes.c_void_p(a) if a else None
+    def call(W=0x1000, s=0x2000, N_src=4, K=256, r=rows, N=3):
+        return L.spense_pack_rows(v(W), v(s), N_src, K, r, N, None, None, 0, 0, None, ctypes.byref(out))
+    assert call(W=0) == 1 and out.value is None
+    assert call(r=None) == 1
+    assert call(N_src=0) == 2 and call(N=0) == 2 and call(K=250) == 2
+    assert call(W=0x1004) == 3
+    assert call() == 1  # rows[1] = 5 is outside [0, 4)
+    assert b"rows[1]" in L.spense_last_error()

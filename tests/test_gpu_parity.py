@@ -270,15 +270,28 @@ def test_grouped_attn32b_qkv(M):
         _assert_close(Y[:, torch.from_numpy(rows).cuda()], yref, bound, f"qkv member {i} M={M}")
 
 
-def test_grouped_rejects_mismatched_layouts():
+def test_grouped_layout_rules():
+    """Members with tail dense sets may differ in Kd (each output is its own
+    GEMM); a different K or a different scattered dense set cannot share X."""
     K = 512
     W, s_w = synth.quantize_rows(synth.normal(77, 1, (128, K), 0.02))
+    X, s_x = synth.quantize_rows(synth.normal(77, 2, (4, K), 1.0))
     a = spense.pack(_dev(W), _dev(s_w), Kd=128)
     b = spense.pack(_dev(W), _dev(s_w), Kd=256)
-    X, s_x = synth.quantize_rows(synth.normal(77, 2, (4, K), 1.0))
-    with pytest.raises(spense.SpenseError) as ei:
-        spense.gemm_grouped([a, b], _dev(X), _dev(s_x), workspace=spense.new_workspace(1 << 20))
-    assert ei.value.code == 1
+    Ya, Yb = spense.gemm_grouped([a, b], _dev(X), _dev(s_x), workspace=spense.new_workspace(1 << 20))
+    torch.cuda.synchronize()
+    for Y, Kd in ((Ya, 128), (Yb, 256)):
+        keep = oracle.pack(W, Kd=Kd)["keep"]
+        yref, bound = oracle.gemm(X, s_x, W, s_w, keep=keep)
+        assert oracle.within_tolerance(Y.float().cpu().numpy(), yref, bound).all()
+    W2, s2 = synth.quantize_rows(synth.normal(77, 3, (128, K + 16), 0.02))
+    c = spense.pack(_dev(W2), _dev(s2), Kd=128)
+    d1 = spense.pack(_dev(W), _dev(s_w), dense_idx=np.arange(0, 256, 2, dtype=np.int32))
+    d2 = spense.pack(_dev(W), _dev(s_w), dense_idx=np.arange(1, 256, 2, dtype=np.int32))
+    for grp in ([a, c], [d1, d2], [a, d1]):
+        with pytest.raises(spense.SpenseError) as ei:
+            spense.gemm_grouped(grp, _dev(X), _dev(s_x), workspace=spense.new_workspace(1 << 20))
+        assert ei.value.code == 1
 
 
 def test_gemm_rejects_small_workspace_and_bad_token_count():
