@@ -44,10 +44,11 @@ def parse():
     ap.add_argument("--dense-frac", type=float, default=0.25)
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--op", choices=["gemm", "quantize", "score"], default="gemm",
+    ap.add_argument("--op", choices=["gemm", "quantize", "score", "glu"], default="gemm",
                     help="gemm: the hybrid GEMM (default, the headline); quantize: the per-token FP8 "
                          "quantisation with the SpenseGPT+ column order fused in; score: the SpenseGPT+ "
-                         "dense-set scorer and top-Kd selection")
+                         "dense-set scorer and top-Kd selection; glu: a 32B-class GLU MLP's three projections "
+                         "under the pages' GLU policy (gate/up output-split, down input-split, permutation folded)")
     return ap.parse_args()
 
 
@@ -657,6 +658,102 @@ def run_score(args):
     return 0
 
 
+def run_glu(args):
+    """The GEMMs of one 32B-class GLU MLP at decode (hidden 5120, intermediate
+    25600) under the pages' GLU policy: gate and up output-split (their dense
+    rows are the SpenseGPT+ dense set, folded to the end of the intermediate
+    order), four members in one launch; down input-split with the same dense
+    set, reading the already-permuted activations without a gather. One step =
+    those two launches (the activation between them is outside this library;
+    a fixed quantised input stands in for it). Timed beside it: the all
+    input-split layout (gate+up as one K-split matrix, down with a tail set)."""
+    import torch
+    from dense_fp8_gemm_b200 import spense, synth, workloads
+    import oracle
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    H, I, M = 5120, 25600, args.tokens
+    Nd = int(round(args.dense_frac * I / 128)) * 128
+    Ns = I - Nd
+    layers = 2
+    D = synth.scored_dense_idx(2, 5, I, Nd)
+    pi = oracle.glu_order(I, D)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    sets, base = [], []
+    for L in range(layers):
+        gq, gs = synth.quantize_rows(synth.normal(2, 40 + L, (I, H), 0.02))
+        uq, us = synth.quantize_rows(synth.normal(2, 50 + L, (I, H), 0.02))
+        dq, ds = synth.quantize_rows(synth.normal(2, 60 + L, (H, I), 0.02))
+        gu = [spense.pack(t(gq), t(gs), Kd=0, rows=pi[:Ns]), spense.pack(t(gq), t(gs), Kd=H, rows=pi[Ns:]),
+              spense.pack(t(uq), t(us), Kd=0, rows=pi[:Ns]), spense.pack(t(uq), t(us), Kd=H, rows=pi[Ns:])]
+        dn = spense.pack(t(dq), t(ds), Kd=Nd, dense_idx=D)
+        sets.append((gu, dn))
+        both = np.concatenate([gq, uq])
+        both_s = np.concatenate([gs, us])
+        base.append((spense.pack(t(both), t(both_s), Kd=workloads.dense_count(H, args.dense_frac)),
+                     spense.pack(t(dq), t(ds), Kd=workloads.dense_count(I, args.dense_frac))))
+        del gq, uq, dq, both
+    x, sx = synth.quantize_rows(synth.normal(2, 70, (M, H), 1.0))
+    h, sh = synth.quantize_rows(synth.normal(2, 71, (M, I), 1.0))
+    X, SX, Hq, SH = t(x), t(sx), t(h), t(sh)
+    G = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+    U = torch.empty((M, I), dtype=torch.bfloat16, device=dev)
+    GU = torch.empty((M, 2 * I), dtype=torch.bfloat16, device=dev)
+    Y = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+    ws = spense.new_workspace(max(spense.grouped_workspace_size(sets[0][0], M), spense.workspace_size(sets[0][1], M),
+                                  spense.workspace_size(base[0][0], M), spense.workspace_size(base[0][1], M)), dev)
+    Ys_gu = [G[:, :Ns], G[:, Ns:], U[:, :Ns], U[:, Ns:]]
+
+    def step_policy(i, st):
+        gu, dn = sets[i % layers]
+        spense.gemm_grouped(gu, X, SX, Ys=Ys_gu, workspace=ws, stream=st)
+        spense.gemm_grouped([dn], Hq, SH, Ys=[Y], workspace=ws, stream=st, flags=spense.GEMM_X_PACKED_ORDER)
+
+    def step_base(i, st):
+        gu, dn = base[i % layers]
+        spense.gemm_grouped([gu], X, SX, Ys=[GU], workspace=ws, stream=st)
+        spense.gemm_grouped([dn], Hq, SH, Ys=[Y], workspace=ws, stream=st)
+
+    mem_gu = [(Ns, H, 0), (Nd, H, H), (Ns, H, 0), (Nd, H, H)]
+    bytes_policy = workloads.group_algorithmic_bytes(mem_gu, M) + workloads.algorithmic_bytes(H, I, Nd, M)
+    kd_h, kd_i = workloads.dense_count(H, args.dense_frac), workloads.dense_count(I, args.dense_frac)
+    bytes_base = workloads.algorithmic_bytes(2 * I, H, kd_h, M) + workloads.algorithmic_bytes(H, I, kd_i, M)
+    steps = max(40, min(args.steps // 20, 1000))
+    with ClockSampler(0) as clocks:
+        t0w = time.time()
+        t_pol, n = graph_time(step_policy, layers, steps, args.warmup // 10)
+        t_base, _ = graph_time(step_base, layers, steps, args.warmup // 10)
+        clocks.mark(t0w, time.time())
+    assert spense.workspace_status(ws) == 0
+    peak, peak_kind = read_peaks()
+    line = {
+        "metric": "spense_glu_mlp_GBps", "value": bytes_policy / t_pol / 1e9, "unit": "GB/s", "n_gpus": 1,
+        "steps": n, "warmup": args.warmup // 10, "ms_per_step": t_pol * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3xe4m3->f32", "data": "synthetic",
+        "config": {"workload": f"32B GLU MLP decode M={M}: gate/up {I}x{H} output-split ({Nd} dense rows, "
+                               f"SpenseGPT+ set folded to the end), down {H}x{I} input-split with the same set, "
+                               f"no gather", "l2": f"{layers} layers rotated (larger than L2)",
+                   "launches_per_step": 2},
+        "input_split_layout": {"GBps": bytes_base / t_base / 1e9, "ms_per_step": t_base * 1e3,
+                               "bytes_per_step": bytes_base},
+        "roofline": {"bound": "hbm", "achieved": bytes_policy / t_pol / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": bytes_policy / t_pol / 1e9 / peak, "traffic": None, "peak_source": peak_kind,
+                     "kernel": "spense_gemm_kernel", "bytes_per_step": bytes_policy},
+        "cpu_baseline": None,
+        "e2e": None,
+        "gpu_launches": 2 * n,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    for gu, dn in sets:
+        for pw in gu + [dn]:
+            pw.free()
+    for a, b in base:
+        a.free()
+        b.free()
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -665,6 +762,8 @@ def main():
         return run_quantize(args)
     if args.op == "score":
         return run_score(args)
+    if args.op == "glu":
+        return run_glu(args)
     return run_spense(args)
 
 
