@@ -154,11 +154,12 @@ __global__ void __launch_bounds__(kScoreThreads) score_finish_kernel(const float
 }
 
 // Top-Kd selection in one CTA: a four-pass radix select over the score bits
-// (non-negative floats order like their bit patterns) finds the Kd-th largest
-// value T; then every score above T and the lowest indices among the scores
-// equal to T are kept, written in ascending index order: each thread owns a
-// contiguous segment of indices, one block-wide scan of its (above, equal)
-// counts gives where its kept indices go.
+// (non-negative floats order like their bit patterns, counted in one
+// histogram per warp) finds the Kd-th largest value T; then every score above
+// T and the lowest indices among the scores equal to T are kept, written in
+// ascending index order: each thread owns a contiguous segment of indices,
+// one block-wide scan of its (above, equal) counts gives where its kept
+// indices go.
 constexpr int kSelectThreads = 1024;
 
 // Exclusive block-wide prefix sum of a 64-bit value (all threads call it).
@@ -191,10 +192,24 @@ __global__ void __launch_bounds__(kSelectThreads) select_top_kernel(const float*
                                                                     int64_t Kd, int32_t* __restrict__ out) {
   extern __shared__ float score_s[];  // kStaged: the I scores
   if (kStaged) {
-    for (int64_t t = threadIdx.x; t < I; t += kSelectThreads) score_s[t] = __ldg(score_g + t);
+    // eight loads in flight per thread: one CTA has to pull the whole array
+    for (int64_t t0 = threadIdx.x; t0 < I; t0 += 8 * kSelectThreads) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t t = t0 + static_cast<int64_t>(u) * kSelectThreads;
+        v[u] = t < I ? __ldg(score_g + t) : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t t = t0 + static_cast<int64_t>(u) * kSelectThreads;
+        if (t < I) score_s[t] = v[u];
+      }
+    }
   }
   const float* score = kStaged ? score_s : score_g;
   __shared__ unsigned int hist[256];
+  __shared__ unsigned int whist[kSelectThreads / 32][256];  // one histogram per warp
   __shared__ uint32_t s_prefix, s_mask;
   __shared__ int64_t s_need;
   __shared__ uint64_t warp_tot[kSelectThreads / 32];
@@ -205,20 +220,18 @@ __global__ void __launch_bounds__(kSelectThreads) select_top_kernel(const float*
     s_need = Kd;  // rank (from the top, 1-based) of T among the scores matching the prefix
   }
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int bb = threadIdx.x; bb < 256; bb += kSelectThreads) hist[bb] = 0u;
+    for (int bb = lane; bb < 256; bb += 32) whist[warp][bb] = 0u;
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
     for (int64_t t = threadIdx.x; t < I; t += kSelectThreads) {
       const uint32_t u = __float_as_uint(score[t]);
-      const bool in = (u & mask) == prefix;
-      // one atomic per distinct bin per warp (scores of similar size share
-      // their high bits, so most of a warp hits the same bin)
-      const unsigned int active = __ballot_sync(__activemask(), in);
-      if (in) {
-        const uint32_t bin = (u >> shift) & 0xFFu;
-        const unsigned int peers = __match_any_sync(active, bin);
-        if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], static_cast<unsigned int>(__popc(peers)));
-      }
+      if ((u & mask) == prefix) atomicAdd(&whist[warp][(u >> shift) & 0xFFu], 1u);
+    }
+    __syncthreads();
+    for (int bb = threadIdx.x; bb < 256; bb += kSelectThreads) {
+      unsigned int c = 0;
+      for (int w = 0; w < kSelectThreads / 32; ++w) c += whist[w][bb];
+      hist[bb] = c;
     }
     __syncthreads();
     if (warp == 0) {
