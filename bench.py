@@ -394,30 +394,45 @@ def run_spense(args):
     peak, peak_kind = read_peaks()
     del g_ev, evs
 
-    # ---- e2e: host buffers in, host buffers out, copies inside the timed region
-    hx = {k: (torch.from_numpy(v[0]).pin_memory(), torch.from_numpy(v[1]).pin_memory()) for k, v in host_x.items()}
-    hy = [torch.empty((M, n), dtype=torch.bfloat16).pin_memory() for _, n, _ in SHAPES]
+    # ---- e2e: host buffers in, host buffers out, copies inside the timed region.
+    # Each group's X and x_scale sit in one pinned host buffer and one device
+    # buffer (one host-to-device copy per group); all outputs of a step sit in
+    # one device buffer (one device-to-host copy per step); the GEMM calls are
+    # prepared once per layer (their arguments marshalled once).
+    import torch as _t
+    in_host, in_dev, in_views = {}, {}, {}
+    for k, (xh, sxh) in host_x.items():
+        nx = xh.size
+        buf_h = _t.empty(nx + 4 * M, dtype=_t.uint8).pin_memory()
+        buf_h[:nx] = _t.from_numpy(xh.reshape(-1))
+        buf_h[nx:] = _t.from_numpy(sxh.view(np.uint8))
+        buf_d = _t.empty_like(buf_h, device=dev)
+        in_host[k], in_dev[k] = buf_h, buf_d
+        in_views[k] = (buf_d[:nx].view(M, -1), buf_d[nx:].view(_t.float32))
+    offs = np.cumsum([0] + [M * n for _, n, _ in SHAPES])
+    out_dev = _t.empty(int(offs[-1]), dtype=_t.bfloat16, device=dev)
+    out_host = _t.empty(int(offs[-1]), dtype=_t.bfloat16).pin_memory()
+    y_views = [out_dev[int(offs[i]):int(offs[i + 1])].view(M, SHAPES[i][1]) for i in range(len(SHAPES))]
+    calls = [[spense.PreparedGrouped([layer[i] for i in grp], in_views[grp[0]][0], in_views[grp[0]][1],
+                                     [y_views[i] for i in grp], ws) for grp in GROUPS] for layer in layers_sp]
     stream = torch.cuda.current_stream()
 
-    def e2e_step(packs):
-        for grp in GROUPS:
-            X, sx = dev_x[grp[0]]
-            X.copy_(hx[grp[0]][0], non_blocking=True)
-            sx.copy_(hx[grp[0]][1], non_blocking=True)
-            spense.gemm_grouped([packs[i] for i in grp], X, sx, [Ys[i] for i in grp], ws, stream)
-            for i in grp:
-                hy[i].copy_(Ys[i], non_blocking=True)
+    def e2e_step(layer_calls):
+        for grp, call in zip(GROUPS, layer_calls):
+            in_dev[grp[0]].copy_(in_host[grp[0]], non_blocking=True)
+            call(stream)
+        out_host.copy_(out_dev, non_blocking=True)
         stream.synchronize()
 
     e2e_steps = max(4, min(args.steps, 200))
     for i in range(min(args.warmup, 8)):
-        e2e_step(layers_sp[i % args.layers])
+        e2e_step(calls[i % args.layers])
     replicas.barrier(ranks)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(e2e_steps):
-        e2e_step(layers_sp[i % args.layers])
+        e2e_step(calls[i % args.layers])
     e1.record()
     torch.cuda.synchronize()
     t_e2e = replicas.max_over_ranks(ranks, [e0.elapsed_time(e1) / 1e3], device=dev)[0]

@@ -2,6 +2,7 @@
 // launch planning (tile, token padding, stream-K grid, pipeline depth), the
 // activation tensor map, and the workspace layout.
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstdlib>
@@ -18,6 +19,7 @@
 using namespace spense;
 
 struct spense_packed {
+  uint64_t id = 0;  // unique for the life of the process (keys the launch cache)
   int device = -1;
   int64_t N = 0, K = 0, Ks = 0, Kd = 0;
   int n_tiles = 0, nsb = 0, ndb = 0;
@@ -376,21 +378,36 @@ spense_status check_gemm_args(const spense_packed* const* hs, int count, int64_t
   return SPENSE_OK;
 }
 
-// Enqueue one launch over `count` packed weights sharing X (arguments validated).
-spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t* X, const float* x_scale,
-                       int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream,
-                       bool x_packed_order = false, const int64_t* ldy = nullptr) {
+// Everything one launch needs, computed once per distinct call (see the
+// launch cache in spense_gemm_grouped_ex).
+struct PreparedLaunch {
+  CUtensorMap map;
+  GemmParams p;
+  uint32_t smem = 0;
+  const uint8_t* gather_src = nullptr;  // SpenseGPT+ gather into gather_dst first, when set
+  const int32_t* perm = nullptr;
+  uint8_t* gather_dst = nullptr;
+  int64_t M = 0, K = 0;
+};
+
+// Builds the launch over `count` packed weights sharing X (arguments validated).
+spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint8_t* X, const float* x_scale,
+                           int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, bool x_packed_order,
+                           const int64_t* ldy, PreparedLaunch* out) {
   const spense_packed* h0 = hs[0];
   const uint8_t* xsrc = X;
+  out->gather_src = nullptr;
   if (h0->perm != nullptr && !x_packed_order) {
-    uint8_t* xg = ws + pl.ws.xg_off;
-    cudaError_t e = launch_gather(X, h0->perm, M, h0->K, xg, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
-    xsrc = xg;
+    out->gather_src = X;
+    out->perm = h0->perm;
+    out->gather_dst = ws + pl.ws.xg_off;
+    out->M = M;
+    out->K = h0->K;
+    xsrc = out->gather_dst;
   }
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return fail(SPENSE_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  CUtensorMap map;
+  CUtensorMap& map = out->map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(h0->K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(h0->K)};
   const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(pl.box_rows)};
@@ -400,7 +417,8 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SPENSE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
 
-  GemmParams p{};
+  GemmParams& p = out->p;
+  p = GemmParams{};
   int tile_begin = 0;
   for (int i = 0; i < count; ++i) {
     GemmMember& m = p.mem[i];
@@ -445,10 +463,63 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
   // the workspace, which nothing sets, so every launch ends by timeout.
   static const bool stall = env_int("SPENSE_TEST_STALL", 0, 0, 1) == 1;
   p.test_gate = stall ? reinterpret_cast<const unsigned int*>(ws + 64) : nullptr;
-  cudaError_t e = launch_gemm(map, p, pl.smem_bytes, stream);
+  out->smem = pl.smem_bytes;
+  return SPENSE_OK;
+}
+
+spense_status enqueue_gemm(const PreparedLaunch& L, cudaStream_t stream) {
+  if (L.gather_src != nullptr) {
+    cudaError_t e = launch_gather(L.gather_src, L.perm, L.M, L.K, L.gather_dst, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "gather launch");
+  }
+  cudaError_t e = launch_gemm(L.map, L.p, L.smem, stream);
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return SPENSE_OK;
 }
+
+// Enqueue one launch over `count` packed weights sharing X (arguments validated).
+spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t* X, const float* x_scale,
+                       int64_t M, uint16_t* const* Ys, uint8_t* ws, const GemmPlan& pl, cudaStream_t stream,
+                       bool x_packed_order = false, const int64_t* ldy = nullptr) {
+  PreparedLaunch L;
+  spense_status st = prepare_gemm(hs, count, X, x_scale, M, Ys, ws, pl, x_packed_order, ldy, &L);
+  if (st != SPENSE_OK) return st;
+  return enqueue_gemm(L, stream);
+}
+
+// Launch cache: repeated calls with the same weights, shapes, pointers and
+// workspace (a decode loop) reuse the plan, the parameter block and the
+// tensor map instead of building them again. Keyed by the handles' unique
+// ids, so a freed and reallocated handle never matches an old entry.
+struct LaunchKey {
+  int device = -1, count = 0;
+  uint64_t ids[kMaxGroup] = {};
+  int64_t M = 0;
+  const void* X = nullptr;
+  const void* x_scale = nullptr;
+  const void* Ys[kMaxGroup] = {};
+  int64_t ldy[kMaxGroup] = {};
+  const void* ws = nullptr;
+  unsigned int flags = 0;
+  bool operator==(const LaunchKey& o) const {
+    if (device != o.device || count != o.count || M != o.M || X != o.X || x_scale != o.x_scale || ws != o.ws ||
+        flags != o.flags)
+      return false;
+    for (int i = 0; i < count; ++i)
+      if (ids[i] != o.ids[i] || Ys[i] != o.Ys[i] || ldy[i] != o.ldy[i]) return false;
+    return true;
+  }
+};
+
+struct LaunchCacheEntry {
+  LaunchKey key;
+  size_t ws_needed = 0;
+  PreparedLaunch launch;
+};
+
+constexpr size_t kLaunchCacheSize = 32;
+std::mutex g_launch_mu;
+std::vector<LaunchCacheEntry>* g_launch_cache = new std::vector<LaunchCacheEntry>();  // most recent first
 
 // ---------------------------------------------------------------- allocation-free entry point
 // Scratch for spense_gemm_noalloc: a fixed array in device memory that every
@@ -555,6 +626,8 @@ spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int
 
   spense_packed* h = new (std::nothrow) spense_packed();
   if (h == nullptr) return fail(SPENSE_ERR_OOM, "host allocation failed");
+  static std::atomic<uint64_t> next_id{1};
+  h->id = next_id.fetch_add(1);
   h->device = dev;
   h->N = N;
   h->K = K;
@@ -681,15 +754,58 @@ spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count,
   DeviceInfo info;
   spense_status st = check_gemm_args(Wps, count, M, workspace, &info);
   if (st != SPENSE_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(SPENSE_ERR_UNSUPPORTED, "no CUDA device");
+  LaunchKey key;
+  key.device = dev;
+  key.count = count;
+  for (int i = 0; i < count; ++i) {
+    if (Wps[i] == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
+    key.ids[i] = Wps[i]->id;
+    key.Ys[i] = Ys[i];
+    key.ldy[i] = ldy != nullptr ? ldy[i] : Wps[i]->N;
+  }
+  key.M = M;
+  key.X = X;
+  key.x_scale = x_scale;
+  key.ws = workspace;
+  key.flags = flags;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  {
+    std::lock_guard<std::mutex> lk(g_launch_mu);
+    auto& cache = *g_launch_cache;
+    for (size_t i = 0; i < cache.size(); ++i) {
+      if (!(cache[i].key == key)) continue;
+      if (workspace_bytes < cache[i].ws_needed)
+        return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                    cache[i].ws_needed);
+      if (i != 0) std::rotate(cache.begin(), cache.begin() + static_cast<std::ptrdiff_t>(i),
+                              cache.begin() + static_cast<std::ptrdiff_t>(i) + 1);
+      st = enqueue_gemm(cache[0].launch, stream);
+      return st == SPENSE_OK ? ok() : st;
+    }
+  }
   GemmPlan pl;
   st = make_plan(Wps, count, M, info.sms, &pl);
   if (st != SPENSE_OK) return st;
   if (workspace_bytes < pl.ws.total_device)
     return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
                 pl.ws.total_device);
-  st = run_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
-                static_cast<cudaStream_t>(stream_v), (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u, ldy);
-  return st == SPENSE_OK ? ok() : st;
+  LaunchCacheEntry entry;
+  entry.key = key;
+  entry.ws_needed = pl.ws.total_device;
+  st = prepare_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
+                    (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u, ldy, &entry.launch);
+  if (st != SPENSE_OK) return st;
+  st = enqueue_gemm(entry.launch, stream);
+  if (st != SPENSE_OK) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_launch_mu);
+    auto& cache = *g_launch_cache;
+    cache.insert(cache.begin(), entry);
+    if (cache.size() > kLaunchCacheSize) cache.pop_back();
+  }
+  return ok();
 }
 
 spense_status spense_quantize(const uint16_t* X, int64_t M, int64_t K, const spense_packed* order, uint8_t* Xq,

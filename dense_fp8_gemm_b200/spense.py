@@ -323,6 +323,27 @@ def gemm_grouped(pws, X: torch.Tensor, x_scale: torch.Tensor, Ys=None, workspace
     return Ys
 
 
+class PreparedGrouped:
+    """A grouped GEMM call with its arguments marshalled once (for loops that
+    launch the same GEMM on the same buffers, such as a decode step): calling
+    it makes one C call. The tensors must stay alive and in place."""
+
+    def __init__(self, pws, X: torch.Tensor, x_scale: torch.Tensor, Ys, workspace: torch.Tensor, flags: int = 0):
+        self._keep = (list(pws), X, x_scale, list(Ys), workspace)
+        yarr = (ctypes.c_void_p * len(pws))()
+        for i, Y in enumerate(Ys):
+            yarr[i] = _dev_ptr(Y, torch.bfloat16, f"Y[{i}]").value
+        self._fn = lib().spense_gemm_grouped_ex
+        self._args = (_handles(pws), len(pws), _dev_ptr(X, torch.uint8, "X"),
+                      _dev_ptr(x_scale, torch.float32, "x_scale"), X.shape[0], yarr, None,
+                      _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), int(flags))
+
+    def __call__(self, stream=None):
+        code = self._fn(*self._args, _stream(stream))
+        if code != SPENSE_OK:
+            _check(code, "spense_gemm_grouped_ex")
+
+
 def quantize(X: torch.Tensor, order: PackedWeight | None = None, Xq: torch.Tensor | None = None,
              x_scale: torch.Tensor | None = None, stream=None):
     """spense_quantize: per-token FP8 quantisation of bf16 activations X [M, K]

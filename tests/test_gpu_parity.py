@@ -308,3 +308,28 @@ def test_gemm_rejects_small_workspace_and_bad_token_count():
         spense.gemm(pw, empty, _dev(s_x[:0]), Y=torch.empty((1, N), dtype=torch.bfloat16, device="cuda"),
                     workspace=spense.new_workspace(need))
     assert ei.value.code == 2
+
+
+def test_launch_cache_follows_handles_and_buffers():
+    """Repeated calls reuse a cached launch; a freed and re-packed weight (which
+    may land at the same address) and changed outputs are never served from a
+    stale entry."""
+    M, N, K, Kd = 8, 256, 512, 128
+    X, s_x, W1, s_w1, _ = _make(61, M, N, K, Kd)
+    _, _, W2, s_w2, _ = _make(62, M, N, K, Kd)
+    Xd, sxd = _dev(X), _dev(s_x)
+    ws = spense.new_workspace(1 << 22)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for W, s_w in ((W1, s_w1), (W2, s_w2), (W1, s_w1)):
+        pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd)
+        for _ in range(3):
+            spense.gemm_grouped([pw], Xd, sxd, [Y], ws)
+        torch.cuda.synchronize()
+        yref, bound = oracle.gemm(X, s_x, W, s_w, keep=oracle.pack(W, Kd=Kd)["keep"])
+        _assert_close(Y, yref, bound, "cached launch")
+        Y2 = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        spense.gemm_grouped([pw], Xd, sxd, [Y2], ws)
+        torch.cuda.synchronize()
+        assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16))
+        pw.free()
+    assert spense.workspace_status(ws) == 0
