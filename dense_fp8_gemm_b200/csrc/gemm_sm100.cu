@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       // before its first store.
       int t, j_unused;
       block_tile(p, b0, t, j_unused);
-      const int m_valid = min(p.npad, p.M - (t % p.m_tiles) * kMaxTokenTile);
+      const int m_valid = min(p.npad, p.M - (t % p.m_tiles) * p.npad);
       const uint32_t bytes = static_cast<uint32_t>((p.cluster - 1) * ((m_valid + 15) >> 4)) * kTileRows * 64u;
       ptx::mbar_arrive_expect_tx(ptx::smem_addr(&bars->peer_done), bytes);
     }
@@ -359,7 +359,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         }
       };
       auto issue_x = [&](const BlockWalker& c, uint32_t s) {
-        const int y0 = c.m_tile * kMaxTokenTile;
+        const int y0 = c.m_tile * p.npad;  // token tiles are npad tokens apart
         const uint32_t b_s = smem_base + s * p.stage_bytes + kBlockBytes;
         const uint32_t full = ptx::smem_addr(&bars->full[s]);
         const GemmMember& mb = p.mem[c.member];
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     // 0; g_lo uses slot 1 when its range started in an earlier tile.
     auto finish_tile = [&](int t) {
       const int n_tile = t / p.m_tiles;
-      const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      const int m0 = (t - n_tile * p.m_tiles) * p.npad;
       stage_sx(m0);
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
@@ -581,7 +581,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       int t, j0, j1;
       units.get(0, t, j0, j1);
       const int n_tile = t / p.m_tiles;
-      const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      const int m0 = (t - n_tile * p.m_tiles) * p.npad;
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
       const int nchunk = (m_valid + 15) >> 4;
@@ -691,7 +691,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
       const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
       const int n_tile = t / p.m_tiles;
-      const int m0 = (t - n_tile * p.m_tiles) * kMaxTokenTile;
+      const int m0 = (t - n_tile * p.m_tiles) * p.npad;
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
       const int n = (n_tile - mb.tile_begin) * kTileRows + row;

@@ -157,6 +157,15 @@ int l2_prefetch_blocks() {
   static const int v = env_int("SPENSE_L2_PREFETCH", 0, 0, 1 << 20);
   return v;
 }
+// Tokens per token tile (multiple of 16, at most 256); 0 (default) =
+// automatic (see make_plan).
+int token_tile_knob() {
+  static const int v = [] {
+    const int x = env_int("SPENSE_TOKEN_TILE", 0, 0, kMaxTokenTile);
+    return x % 16 == 0 ? x : 0;
+  }();
+  return v;
+}
 int producers() {
   static const int v = env_int("SPENSE_PRODUCERS", 2, 1, 2);
   return v;
@@ -188,16 +197,28 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   const spense_packed* h0 = hs[0];
   if (h0 == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
   GemmPlan pl{};
-  pl.npad = M > kMaxTokenTile ? kMaxTokenTile : static_cast<int>(round_up(static_cast<size_t>(M), 16));
-  pl.box_rows = static_cast<int>(M > kMaxTokenTile ? kMaxTokenTile : M);
-  pl.m_tiles = static_cast<int>((M + kMaxTokenTile - 1) / kMaxTokenTile);
+  long long row_tiles = 0;
+  for (int i = 0; i < count; ++i) {
+    if (hs[i] == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
+    row_tiles += hs[i]->n_tiles;
+  }
+  // Token tile T: all tokens in one tile up to T, else tiles of T tokens. The
+  // CTAs of neighbouring token tiles stream the same weight rows at about the
+  // same time, so the repeat reads hit L2. 64 tokens while the tiles of 64
+  // fit two per SM (a cluster split or a short stream-K range per CTA keeps
+  // every SM streaming), 128 for launches with more tiles than that, where
+  // each CTA owns whole tiles and a wider tile halves the L2 re-reads.
+  const int T = token_tile_knob() != 0 ? token_tile_knob()
+                                       : (row_tiles * ((M + 63) / 64) <= 2LL * sms ? 64 : 128);
+  pl.npad = M > T ? T : static_cast<int>(round_up(static_cast<size_t>(M), 16));
+  pl.box_rows = static_cast<int>(M > T ? T : M);
+  pl.m_tiles = static_cast<int>((M + T - 1) / T);
   pl.count = count;
   long long n_tiles = 0, blocks = 0, cost = 0;
   pl.min_tile_cost = 1 << 30;
   pl.any_sparse = false;
   for (int i = 0; i < count; ++i) {
     const spense_packed* h = hs[i];
-    if (h == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
     if (h->device != h0->device || h->K != h0->K || h->perm_host != h0->perm_host)
       return fail(SPENSE_ERR_ARG,
                   "packed weights sharing a launch need the same device, K and column order of X (the same "
@@ -231,24 +252,66 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.any_sparse ? 256u : 128u);
   pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.any_sparse ? kMetaBlockBytes : 0);
   const uint32_t reserve = 1024 + kBarrierBytes;  // alignment slack + barrier area
-  const int cps_first =
-      ctas_per_sm_knob() != 0 ? ctas_per_sm_knob() : ((pl.tiles > 2 * sms || pl.npad > 32) ? 1 : 2);
-  for (int cps = cps_first; cps >= 1; --cps) {
+  // Ring and TMEM for `cps` CTAs per SM; false if two stages or the
+  // accumulators do not fit.
+  auto fit_ring = [&](int cps, uint32_t recv, int* stages, int* nacc, uint32_t* cols) {
     const uint32_t smem_budget = gemm_max_smem() / cps - (cps > 1 ? 1024u : 0u);
     const uint32_t tmem_budget = 512u / cps;
-    const int stages = static_cast<int>(std::min<uint32_t>(kMaxStages, (smem_budget - reserve) / pl.stage_bytes));
-    const int nacc = (2u * pl.npad + 16u <= tmem_budget) ? 2 : 1;
-    uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(nacc * pl.npad + 16)) cols <<= 1;
-    if ((stages < 2 || cols > tmem_budget) && cps > 1) continue;
-    pl.ctas_per_sm = cps;
-    pl.stages = stages;
-    pl.nacc = nacc;
-    pl.tmem_cols = cols;
-    break;
+    if (smem_budget < reserve + recv + 2 * pl.stage_bytes) return false;
+    *stages = static_cast<int>(std::min<uint32_t>(kMaxStages, (smem_budget - reserve - recv) / pl.stage_bytes));
+    *nacc = (2u * pl.npad + 16u <= tmem_budget) ? 2 : 1;
+    *cols = 32;
+    while (*cols < static_cast<uint32_t>(*nacc * pl.npad + 16)) *cols <<= 1;
+    return *cols <= tmem_budget;
+  };
+  auto slots_for = [&](int cps) {
+    return std::min<long long>(static_cast<long long>(sms) * std::min(cps, grid_per_sm()), kMaxGrid);
+  };
+  // Few tiles (at most half the CTA slots): the CTAs of a cluster of S split
+  // each tile's K range by weight and reduce in shared memory; otherwise
+  // stream-K over all tiles with the global fix-up. Cluster sizes are powers
+  // of two (a grid of clusters of 7 did not fit in one wave); the cluster
+  // grid must fit the CTA slots and fill at least half of them, unless the
+  // GEMM is so small that fixed costs dominate anyway, and rank 0's receive
+  // area (S - 1 partials of 128 rows x npad floats) comes out of the ring.
+  // Returns the largest such S for `cps` CTAs per SM, or 1.
+  const int mode = cluster_mode();
+  auto cluster_for = [&](int cps) {
+    const long long slots = slots_for(cps);
+    if (mode == 0 || pl.tiles * 2 > slots || pl.npad > 64) return 1;
+    for (int S = 8; S >= 2; S >>= 1) {
+      if (mode > 1 && S != mode) continue;
+      if (pl.tiles * S > slots || S > pl.min_tile_cost / kCostSparse) continue;
+      const bool fills = pl.tiles * S * 2 >= slots;
+      const bool small = pl.total_cost < 40LL * slots;
+      if (!(mode > 1 || fills || small)) continue;
+      int st, na;
+      uint32_t co;
+      if (fit_ring(cps, static_cast<uint32_t>(S - 1) * kTileRows * pl.npad * 4u, &st, &na, &co)) return S;
+    }
+    return 1;
+  };
+  // CTAs per SM: two (two independent copy streams that hide each other's
+  // fixed costs) when the launch has at most two row tiles per SM and the
+  // token tile is at most 32 tokens, else one with a deeper ring. A launch
+  // that cannot split its tiles over clusters at that count but can at the
+  // other count takes the other.
+  const int knob = ctas_per_sm_knob();
+  int cps = knob != 0 ? knob : ((pl.tiles > 2 * sms || pl.npad > 32) ? 1 : 2);
+  pl.cluster = cluster_for(cps);
+  if (pl.cluster == 1 && knob == 0 && cluster_for(3 - cps) > 1) {
+    cps = 3 - cps;
+    pl.cluster = cluster_for(cps);
   }
-  const long long slots =
-      std::min<long long>(static_cast<long long>(sms) * std::min(pl.ctas_per_sm, grid_per_sm()), kMaxGrid);
+  pl.recv_bytes = pl.cluster > 1 ? static_cast<uint32_t>(pl.cluster - 1) * kTileRows * pl.npad * 4u : 0u;
+  if (!fit_ring(cps, pl.recv_bytes, &pl.stages, &pl.nacc, &pl.tmem_cols)) {
+    // Stream-K (no receive area) and two CTAs per SM that do not fit: one.
+    cps = 1;
+    if (!fit_ring(cps, 0, &pl.stages, &pl.nacc, &pl.tmem_cols))
+      return fail(SPENSE_ERR_SHAPE, "token tile of %d does not fit one CTA", pl.npad);
+  }
+  pl.ctas_per_sm = cps;
+  const long long slots = slots_for(cps);
   // First block of a tile of member i whose start weight is >= c (c within one tile).
   auto block_at = [&](int i, long long c) {
     const long long sp = static_cast<long long>(kCostSparse) * pl.mem_nsb[i];
@@ -271,41 +334,6 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     for (int k = 0; k < i; ++k) first_tile += static_cast<long long>(pl.mem_tiles[k]) * pl.m_tiles;
     return pl.mem_block_begin[i] + (t - first_tile) * (pl.mem_nsb[i] + pl.mem_ndb[i]);
   };
-  // Few tiles (at most half the CTA slots): the CTAs of a cluster of S split
-  // each tile's K range by weight and reduce in shared memory; otherwise
-  // stream-K over all tiles with the global fix-up.
-  pl.cluster = 1;
-  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes;
-  const int mode = cluster_mode();
-  if (mode != 0 && pl.tiles * 2 <= slots && pl.npad <= 64) {
-    // Power-of-two cluster sizes (a grid of clusters of 7 did not fit in one
-    // wave); the cluster grid must fit the CTA slots and fill at least half of
-    // them, unless the GEMM is so small that fixed costs dominate anyway.
-    for (int S = 8; S >= 2; S >>= 1) {
-      if (mode > 1 && S != mode) continue;
-      if (pl.tiles * S > slots || S > pl.min_tile_cost / kCostSparse) continue;
-      const bool fills = pl.tiles * S * 2 >= slots;
-      const bool small = pl.total_cost < 40LL * slots;
-      if (mode > 1 || fills || small) {
-        pl.cluster = S;
-        break;
-      }
-    }
-  }
-  pl.recv_bytes = 0;
-  if (pl.cluster > 1) {
-    // Rank 0 receives S - 1 partials of 128 rows x npad floats; the ring gives
-    // up stages for it (at least two must remain).
-    pl.recv_bytes = static_cast<uint32_t>(pl.cluster - 1) * kTileRows * pl.npad * 4u;
-    const uint32_t smem_budget = gemm_max_smem() / pl.ctas_per_sm - (pl.ctas_per_sm > 1 ? 1024u : 0u);
-    if (smem_budget < reserve + pl.recv_bytes + 2 * pl.stage_bytes) {
-      pl.cluster = 1;
-      pl.recv_bytes = 0;
-    } else {
-      pl.stages = static_cast<int>(
-          std::min<uint32_t>(kMaxStages, (smem_budget - reserve - pl.recv_bytes) / pl.stage_bytes));
-    }
-  }
   if (pl.cluster > 1) {
     pl.grid = pl.tiles * pl.cluster;
     for (int g = 0; g <= pl.grid; ++g) {
