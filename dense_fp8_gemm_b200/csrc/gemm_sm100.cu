@@ -35,9 +35,9 @@
 // CTA order, so the result does not depend on arrival order.
 //
 // Launches with few tiles use a cluster split instead: the S CTAs of a cluster
-// (S = 2, 4 or 8) stream consecutive K ranges of one tile; the peers send
-// their fp32 partials into rank 0's shared memory with asynchronous
-// distributed-shared-memory stores, and rank 0 adds them in rank order.
+// (S = 2, 4 or 8) stream consecutive K ranges of one tile; each peer stages
+// its fp32 partial in its idle ring and sends it into rank 0's shared memory
+// with one shared-to-shared bulk copy, and rank 0 adds them in rank order.
 //
 // Every wait is bounded (1.5 s by %globaltimer); on expiry the kernel records a
 // code in the workspace status word and all roles leave their loops.

@@ -197,19 +197,22 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   const spense_packed* h0 = hs[0];
   if (h0 == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
   GemmPlan pl{};
-  long long row_tiles = 0;
+  long long row_tiles = 0, weight_units = 0;
   for (int i = 0; i < count; ++i) {
     if (hs[i] == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
     row_tiles += hs[i]->n_tiles;
+    weight_units += static_cast<long long>(hs[i]->n_tiles) * (kCostSparse * hs[i]->nsb + kCostDense * hs[i]->ndb);
   }
   // Token tile T: all tokens in one tile up to T, else tiles of T tokens. The
   // CTAs of neighbouring token tiles stream the same weight rows at about the
   // same time, so the repeat reads hit L2. 64 tokens while the tiles of 64
-  // fit two per SM (a cluster split or a short stream-K range per CTA keeps
-  // every SM streaming), 128 for launches with more tiles than that, where
-  // each CTA owns whole tiles and a wider tile halves the L2 re-reads.
+  // fit one per SM (they then split over clusters), or two per SM for a
+  // weight of at most 32 MB (its repeat reads stay in L2); 128 otherwise,
+  // which halves the repeat reads and gives each CTA longer whole tiles.
+  const long long tiles64 = row_tiles * ((M + 63) / 64);
+  const bool small_weight = weight_units * 4096ll <= (32ll << 20);  // cost units are 4 KiB
   const int T = token_tile_knob() != 0 ? token_tile_knob()
-                                       : (row_tiles * ((M + 63) / 64) <= 2LL * sms ? 64 : 128);
+                                       : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128);
   pl.npad = M > T ? T : static_cast<int>(round_up(static_cast<size_t>(M), 16));
   pl.box_rows = static_cast<int>(M > T ? T : M);
   pl.m_tiles = static_cast<int>((M + T - 1) / T);
