@@ -58,6 +58,14 @@ SHAPES = (("q_proj", 8192, 5120), ("k_proj", 1024, 5120), ("v_proj", 1024, 5120)
 GROUPS = ((0, 1, 2), (3,))
 
 
+L2_BYTES = 126 << 20
+
+
+def l2_note(sets, total):
+    rel = "larger" if total > L2_BYTES else "NOT larger"
+    return f"{sets} weight sets rotated per step ({total / 1e6:.0f} MB, {rel} than the 126 MB L2)"
+
+
 def workload_config(args):
     return {
         "workload": f"attn32b q/k/v/o projections, decode M={args.tokens}",
@@ -67,7 +75,7 @@ def workload_config(args):
         "dense_frac": args.dense_frac,
         "dense_columns": "tail (SpenseGPT)",
         "weights": "FP8 e4m3 N(0,0.02) per-channel absmax scales; X N(0,1) per-token scales; seed 1",
-        "l2": f"{args.layers} weight sets rotated per step (inputs larger than L2)",
+        "l2": l2_note(args.layers, args.layers * step_bytes(args)),
         "graph": f"one CUDA graph per {args.layers} steps (the rotated layers back to back)",
     }
 

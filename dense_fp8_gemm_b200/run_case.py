@@ -2,17 +2,23 @@
 
     python -m dense_fp8_gemm_b200.run_case --workload attn32b --tokens 16 --repeat 3
     python -m dense_fp8_gemm_b200.run_case --shape 51200x5120 --dense-frac 0.25 --tokens 16 --repeat 3
+    python -m dense_fp8_gemm_b200.run_case --shape 5120x25600 --scattered --tokens 8192 --repeat 1
+    python -m dense_fp8_gemm_b200.run_case --shape 25600x5120 --output-split --tokens 16 --repeat 1
 
 `attn32b` issues, per repeat, the two launches of one decoder layer's attention
 projections: q, k and v grouped on one input, then o_proj. `--shape NxK` runs a
-single GEMM. Every launch goes through the C ABI; inputs are seeded synthetic
-tensors (see synth.py).
+single GEMM: with `--scattered` its dense columns are a seeded random set
+(SpenseGPT+, so each call gathers X into the packed column order first); with
+`--output-split` its 2:4 rows and its dense rows (a seeded random set) are
+packed as two weights (spense_pack_rows) that share one launch. Every launch
+goes through the C ABI; inputs are seeded synthetic tensors (see synth.py).
 """
 from __future__ import annotations
 
 import argparse
 import sys
 
+import numpy as np
 import torch
 
 from . import spense, synth, workloads
@@ -25,6 +31,8 @@ def main(argv=None):
     ap.add_argument("--dense-frac", type=float, default=0.25)
     ap.add_argument("--tokens", type=int, default=16)
     ap.add_argument("--repeat", type=int, default=3)
+    ap.add_argument("--scattered", action="store_true", help="SpenseGPT+ dense column set (seeded)")
+    ap.add_argument("--output-split", action="store_true", help="2:4 rows and dense rows packed apart")
     args = ap.parse_args(argv)
     dev = torch.device("cuda")
     M = args.tokens
@@ -38,10 +46,20 @@ def main(argv=None):
     if args.shape is not None:
         N, K = (int(v) for v in args.shape.lower().split("x"))
         W, s_w = synth.quantize_rows(synth.normal(1, 2, (N, K), 0.02))
-        pw = spense.pack(torch.from_numpy(W).to(dev), torch.from_numpy(s_w).to(dev),
-                         Kd=workloads.dense_count(K, args.dense_frac))
+        Wd, sd = torch.from_numpy(W).to(dev), torch.from_numpy(s_w).to(dev)
+        Kd = workloads.dense_count(K, args.dense_frac)
+        rng = np.random.default_rng(5)
+        if args.output_split:
+            nd = int(round(args.dense_frac * N / 8)) * 8
+            dense_rows = np.sort(rng.choice(N, nd, replace=False))
+            sparse_rows = np.setdiff1d(np.arange(N), dense_rows)
+            grp = [spense.pack(Wd, sd, Kd=0, rows=sparse_rows), spense.pack(Wd, sd, Kd=K, rows=dense_rows)]
+        elif args.scattered:
+            grp = [spense.pack(Wd, sd, dense_idx=np.sort(rng.choice(K, Kd, replace=False)))]
+        else:
+            grp = [spense.pack(Wd, sd, Kd=Kd)]
         X, s_x = synth.quantize_rows(synth.normal(1, 3, (M, K), 1.0))
-        launches.append(([pw], torch.from_numpy(X).to(dev), torch.from_numpy(s_x).to(dev)))
+        launches.append((grp, torch.from_numpy(X).to(dev), torch.from_numpy(s_x).to(dev)))
     else:
         wl = workloads.ATTN32B
         qkv = [packed(wl, i) for i in range(3)]
