@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   if (threadIdx.x == 0) {
     ptx::prefetch_tensormap(&tmap_x);
     for (int s = 0; s < p.stages; ++s) {
-      ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1);
+      ptx::mbar_init(ptx::smem_addr(&bars->full[s]), 1 + p.x_warp);
       ptx::mbar_init(ptx::smem_addr(&bars->empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -301,42 +301,87 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   const Units units(p, b0, b1);
   const uint32_t smem_base = ptx::smem_addr(smem);
 
-  if (warp == 0 || warp == 6) {
+  // Loader warps: warp 0 (and warp 6 with two weight loaders) copy the weight
+  // blocks; with x_warp the next warp copies the activation tiles.
+  const int x_loader = p.x_warp ? 5 + p.producers : -1;
+  const uint32_t bar2_threads = 32u * static_cast<uint32_t>(p.producers + p.x_warp);
+  // Test of the failure path: every loader waits (bounded) on a word nothing
+  // sets, before any copy is issued, so the timeout leaves no transfer in flight.
+  auto test_gate_wait = [&]() {
+    if (lane != 0 || p.test_gate == nullptr) return;
+    const uint64_t t0 = ptx::globaltimer();
+    while (*reinterpret_cast<const volatile unsigned int*>(p.test_gate) == 0u && !*abort_flag) {
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        atomicOr(p.status, SPENSE_DEVICE_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+        break;
+      }
+      __nanosleep(1000);
+    }
+  };
+
+  if (warp == x_loader) {
+    // ------------------------------------------------------------ activation loader
+    // The activation tile of every block, in the ring's order, as an issue
+    // stream of its own: the copy engine serves each issuing thread's copies
+    // one after another, so these small copies (the MMA needs them, and they
+    // wait for the previous grid) do not queue behind the weight copies.
+    ptx::named_bar_sync(2, bar2_threads);  // the barriers are initialised
+    if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+    test_gate_wait();
+    if (lane == 0 && !*abort_flag) {
+      ptx::griddep_wait();  // X may be written by the previous grid
+      const uint64_t pol_x = ptx::policy_evict_last();
+      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;       // smem bytes of a K-atom
+      const uint32_t xb = static_cast<uint32_t>(p.box_rows) * 128u;    // bytes of one TMA box
+      BlockWalker cx(units, p);
+      Ring ring(static_cast<uint32_t>(p.stages));
+      const int nb = b1 - b0;
+      for (int i = 0; i < nb; ++i, ring.advance(), cx.advance(p)) {
+        if (i >= p.stages && !wait_bar(ptx::smem_addr(&bars->empty[ring.s]), ring.ph ^ 1u, p.status,
+                                       SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag))
+          break;
+        const GemmMember& mb = p.mem[cx.member];
+        const int y0 = cx.m_tile * p.npad;
+        const uint32_t b_s = smem_base + ring.s * p.stage_bytes + kBlockBytes;
+        const uint32_t full = ptx::smem_addr(&bars->full[ring.s]);
+        if (cx.j < mb.nsb) {
+          ptx::mbar_arrive_expect_tx(full, 2 * xb);
+          ptx::tma_load_2d(b_s, &tmap_x, cx.j * kSparseBlockCols, y0, full, pol_x);
+          ptx::tma_load_2d(b_s + box, &tmap_x, cx.j * kSparseBlockCols + 128, y0, full, pol_x);
+        } else {
+          ptx::mbar_arrive_expect_tx(full, xb);
+          ptx::tma_load_2d(b_s, &tmap_x, mb.Ks + (cx.j - mb.nsb) * kDenseBlockCols, y0, full, pol_x);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 0 || (warp == 6 && p.producers > 1)) {
     // ------------------------------------------------------------ producer(s)
     // Blocks go through the ring in processing order. The weight copies of
     // the first ring's worth are issued before waiting on the previous grid
-    // (the packed weights never depend on it), the activation tiles after.
-    // With two producer warps (warps 0 and 6) each issues every other block:
-    // the copy engine serves the two issue streams concurrently.
+    // (the packed weights never depend on it), the activation tiles after
+    // (unless the activation loader issues them). With two producer warps
+    // (warps 0 and 6) each issues every other block: the copy engine serves
+    // the two issue streams concurrently.
     if (warp == 0) {
       __syncwarp();  // lane 0 initialised the barriers
       if (p.cluster > 1) ptx::cluster_arrive_relaxed();
       ptx::named_bar_arrive(3, kGemmThreads);
-      if (p.producers > 1) ptx::named_bar_arrive(2, 64);
+      if (bar2_threads > 32u) ptx::named_bar_arrive(2, bar2_threads);
     } else {
-      ptx::named_bar_sync(2, 64);
+      ptx::named_bar_sync(2, bar2_threads);
       if (p.cluster > 1) ptx::cluster_arrive_relaxed();
     }
-    if (lane == 0 && p.test_gate != nullptr) {
-      // Test of the failure path: wait (bounded) on a word nothing sets, before
-      // any copy is issued, so the timeout leaves no transfer in flight.
-      const uint64_t t0 = ptx::globaltimer();
-      while (*reinterpret_cast<const volatile unsigned int*>(p.test_gate) == 0u) {
-        if (ptx::globaltimer() - t0 > kWaitLimitNs) {
-          atomicOr(p.status, SPENSE_DEVICE_TIMEOUT_PRODUCER);
-          *abort_flag = 1;
-          break;
-        }
-        __nanosleep(1000);
-      }
-    }
+    test_gate_wait();
     if (lane == 0 && !*abort_flag) {
       const int np = p.producers;
       const int me = warp == 0 ? 0 : 1;
       const uint64_t pol_w = ptx::policy_evict_first();
       const uint64_t pol_x = ptx::policy_evict_last();
       const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;         // smem bytes of a K-atom
-      const uint32_t xbytes = static_cast<uint32_t>(p.box_rows) * 128u;  // bytes one TMA box loads
+      // bytes one TMA box of activations loads (none here when the activation loader issues them)
+      const uint32_t xbytes = p.x_warp ? 0u : static_cast<uint32_t>(p.box_rows) * 128u;
       const int nb = b1 - b0;
       const int pre = nb < p.stages ? nb : p.stages;
       auto issue_w = [&](const BlockWalker& c, uint32_t s) {
@@ -392,10 +437,12 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
           }
         }
       }
-      ptx::griddep_wait();
-      BlockWalker cx(units, p);
-      for (int i = 0; i < pre; ++i, cx.advance(p))
-        if (i % np == me) issue_x(cx, static_cast<uint32_t>(i));
+      if (!p.x_warp) {
+        ptx::griddep_wait();
+        BlockWalker cx(units, p);
+        for (int i = 0; i < pre; ++i, cx.advance(p))
+          if (i % np == me) issue_x(cx, static_cast<uint32_t>(i));
+      }
       Ring ring(static_cast<uint32_t>(p.stages));
       for (int i = 0; i < pre; ++i) ring.advance();
       for (int i = pre; i < nb; ++i, ring.advance(), cw.advance(p)) {
@@ -404,7 +451,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
                       SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag))
           break;
         issue_w(cw, ring.s);
-        issue_x(cw, ring.s);
+        if (!p.x_warp) issue_x(cw, ring.s);
       }
     }
   } else if (warp == 1) {
@@ -830,7 +877,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
   }();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned int>(p.grid));
-  cfg.blockDim = dim3(kGemmThreads + 32 * (p.producers - 1));
+  cfg.blockDim = dim3(kGemmThreads + 32 * (p.producers - 1) + 32 * p.x_warp);
   cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[3];

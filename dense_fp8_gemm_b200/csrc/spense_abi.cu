@@ -166,6 +166,12 @@ int token_tile_knob() {
   }();
   return v;
 }
+// 1 (default): a warp of its own issues the activation-tile loads; 0: the
+// weight loaders issue them after the weight copies.
+int x_warp() {
+  static const int v = env_int("SPENSE_X_WARP", 1, 0, 1);
+  return v;
+}
 int producers() {
   static const int v = env_int("SPENSE_PRODUCERS", 2, 1, 2);
   return v;
@@ -490,6 +496,7 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
   p.cluster = pl.cluster;
   p.recv_bytes = pl.recv_bytes;
   p.l2_prefetch = l2_prefetch_blocks();
+  p.x_warp = x_warp();
   // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
   // the workspace, which nothing sets, so every launch ends by timeout.
   static const bool stall = env_int("SPENSE_TEST_STALL", 0, 0, 1) == 1;

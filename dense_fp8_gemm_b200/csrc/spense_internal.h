@@ -19,7 +19,7 @@ constexpr int kMaxTokenTile = 256;      // tokens per tile (MMA N upper bound)
 constexpr int kCostSparse = 5;          // HBM bytes of a sparse block in 4 KiB units (16 + 4 KiB)
 constexpr int kCostDense = 4;           // ... of a dense block (16 KiB)
 constexpr int kGemmThreads = 192;       // warp 0 loads, warp 1 issues MMAs, warps 2-5 epilogue
-constexpr int kGemmThreadsMax = 224;    // plus warp 6 as a second loader
+constexpr int kGemmThreadsMax = 256;    // plus a second weight loader and an activation loader
 constexpr int kMaxStages = 12;
 constexpr uint32_t kBarrierBytes = 2048;  // mbarriers, flags and staged token scales
 
@@ -103,6 +103,7 @@ struct GemmParams {
   const unsigned int* test_gate;  // test only: loaders wait (bounded) until this word is nonzero
   uint32_t recv_bytes;            // cluster mode: rank 0's receive area for the peers' partials
   int l2_prefetch;                // blocks past the first ring's worth prefetched into L2 at start
+  int x_warp;                     // 1: a warp of its own issues the activation-tile loads
 };
 
 // Kernels (defined in the .cu files).
