@@ -15,11 +15,13 @@
 // one activation tensor (for example q, k and v projections); their row tiles
 // are laid end to end.
 //
-// Roles (up to two CTAs per SM, 192 or 224 threads):
+// Roles (up to two CTAs per SM, 192 to 256 threads):
 //   warps 0, 6 producers: bulk copies of the packed weight blocks (values,
-//            metadata, dense columns) and 2-D TMA loads of the activation tile
-//            into a ring of shared-memory stages; with two producer warps
-//            each issues every other block;
+//            metadata, dense columns) into a ring of shared-memory stages;
+//            with two producer warps each issues every other block;
+//   warp 7   (warp 6 with one producer) 2-D TMA loads of the activation tile
+//            of every block into the same stages (without it, the producers
+//            issue them after each stage's weight copies);
 //   warp 1   allocates tensor memory; one lane copies the metadata into tensor
 //            memory (tcgen05.cp) and issues the MMAs;
 //   warps 2-5 epilogue: tensor memory -> registers, scales, bf16 stores, or
