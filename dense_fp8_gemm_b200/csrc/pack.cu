@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cstdint>
 
+#include "pdl.cuh"
 #include "spense_internal.h"
 
 namespace spense {
@@ -181,6 +182,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint8_t* __restr
 __global__ void __launch_bounds__(256) gather_kernel(const uint8_t* __restrict__ X,
                                                      const int32_t* __restrict__ perm, int64_t M,
                                                      int64_t K, uint8_t* __restrict__ Xg) {
+  pdl_trigger();  // the GEMM that reads Xg may start prefetching its weights
+  pdl_wait();     // X may be written by the previous kernel
   const int64_t quads = K / 4;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < M * quads;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -244,8 +247,7 @@ cudaError_t launch_gather(const uint8_t* X, const int32_t* perm, int64_t M, int6
                           cudaStream_t stream) {
   const int64_t threads = M * (K / 4);
   const unsigned int grid = static_cast<unsigned int>(std::min<int64_t>(blocks_for(threads), 4096));
-  gather_kernel<<<grid, 256, 0, stream>>>(X, perm, M, K, Xg);
-  return cudaGetLastError();
+  return launch_pdl(gather_kernel, grid, 256, 0, stream, X, perm, M, K, Xg);
 }
 
 }  // namespace spense

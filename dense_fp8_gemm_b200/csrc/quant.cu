@@ -17,6 +17,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "pdl.cuh"
 #include "spense_internal.h"
 
 namespace spense {
@@ -60,6 +61,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t*
                                                                  int C) {
   extern __shared__ uint4 qsmem[];  // kStaged: the row, K bf16
   __shared__ float red[kQuantThreads / 32];
+  pdl_trigger();  // the GEMM that reads Xq may start prefetching its weights
+  pdl_wait();     // X may be written by the previous kernel
   const int64_t m = blockIdx.x / C;
   const int c = static_cast<int>(blockIdx.x % C);
   const int64_t k16 = K / 16;
@@ -162,15 +165,11 @@ cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32
   while (C > 1 && K / 16 < C) --C;
   const unsigned int grid = static_cast<unsigned int>(M * C);
   const int ci = static_cast<int>(C);
-  if (perm == nullptr) {
-    quantize_kernel<false, false><<<grid, kQuantThreads, 0, stream>>>(X, K, perm, Xq, s_x, ci);
-    return cudaGetLastError();
-  }
+  if (perm == nullptr)
+    return launch_pdl(quantize_kernel<false, false>, grid, kQuantThreads, 0, stream, X, K, perm, Xq, s_x, ci);
   const int64_t stage = K * 2;
-  if (stage > kQuantStageBytes) {
-    quantize_kernel<true, false><<<grid, kQuantThreads, 0, stream>>>(X, K, perm, Xq, s_x, ci);
-    return cudaGetLastError();
-  }
+  if (stage > kQuantStageBytes)
+    return launch_pdl(quantize_kernel<true, false>, grid, kQuantThreads, 0, stream, X, K, perm, Xq, s_x, ci);
   static thread_local int configured_for = -1;
   int dev = 0;
   cudaError_t st = cudaGetDevice(&dev);
@@ -181,8 +180,8 @@ cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32
     if (st != cudaSuccess) return st;
     configured_for = dev;
   }
-  quantize_kernel<true, true><<<grid, kQuantThreads, static_cast<size_t>(stage), stream>>>(X, K, perm, Xq, s_x, ci);
-  return cudaGetLastError();
+  return launch_pdl(quantize_kernel<true, true>, grid, kQuantThreads, static_cast<size_t>(stage), stream, X, K, perm,
+                    Xq, s_x, ci);
 }
 
 }  // namespace spense
