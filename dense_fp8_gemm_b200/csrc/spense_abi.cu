@@ -152,9 +152,12 @@ int grid_per_sm() {
   static const int v = env_int("SPENSE_GRID_PER_SM", 2, 1, 2);
   return v;
 }
-// Blocks per CTA prefetched into L2 at start (0 = none).
-int l2_prefetch_blocks() {
-  static const int v = env_int("SPENSE_L2_PREFETCH", 0, 0, 1 << 20);
+// Weight blocks per CTA, past the first ring's worth, prefetched into L2 at
+// start; -1 (default) = automatic: 4 for cluster-split launches (few tiles;
+// the prefetch overlaps the previous grid's tail: attn32b decode step 0.505
+// -> 0.524 of HBM), none for stream-K launches (gate+up 33.5 -> 34.5 us with 8).
+int l2_prefetch_knob() {
+  static const int v = env_int("SPENSE_L2_PREFETCH", -1, -1, 1 << 20);
   return v;
 }
 // Tokens per token tile (multiple of 16, at most 256); 0 (default) =
@@ -495,7 +498,7 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
   p.producers = pl.producers;
   p.cluster = pl.cluster;
   p.recv_bytes = pl.recv_bytes;
-  p.l2_prefetch = l2_prefetch_blocks();
+  p.l2_prefetch = l2_prefetch_knob() >= 0 ? l2_prefetch_knob() : (pl.cluster > 1 ? 4 : 0);
   p.x_warp = x_warp();
   // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
   // the workspace, which nothing sets, so every launch ends by timeout.
