@@ -125,12 +125,12 @@ long long min_cta_weight() {
 }
 
 // Tuning knobs read once from the environment: CTAs per SM (1, 2 or 0 =
-// automatic), loader warps per CTA (1 or 2, default 2) and how many bulk
-// copies move one 16 KiB weight block (1, 2 or 4, default 1). One SM's copy
-// engine serves several issue streams at once but one stream's copies one
-// after another, so two CTAs with two loader warps each keep four streams
-// going per SM; a single CTA with a ring twice as deep does as well on long
-// GEMMs.
+// automatic), weight-loader warps per CTA (1 or 2, default 2; one more warp
+// loads the activation tiles) and how many bulk copies move one 16 KiB weight
+// block (1, 2 or 4, default 1). One SM's copy engine serves several issue
+// streams at once but one stream's copies one after another, so two CTAs
+// with two weight loaders each keep four weight streams going per SM; a
+// single CTA with a ring twice as deep does as well on long GEMMs.
 int env_int(const char* name, int dflt, int lo, int hi) {
   const char* e = std::getenv(name);
   if (e == nullptr) return dflt;
