@@ -278,9 +278,9 @@ def run_spense(args):
 
     ranks = replicas.from_env()
     world, rank, local = ranks.world, ranks.rank, ranks.local
-    replicas.init(ranks, "nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    replicas.init(ranks, "nccl", device=dev)
 
     M = args.tokens
     wl = workloads.ATTN32B

@@ -26,13 +26,15 @@ def from_env() -> RankInfo:
                     int(os.environ.get("LOCAL_RANK", "0")))
 
 
-def init(info: RankInfo, backend: str, timeout_s: float = 120.0):
+def init(info: RankInfo, backend: str, timeout_s: float = 120.0, device=None):
     """Join the process group when there is more than one rank (short timeout,
-    so ranks that wait for a missing peer fail instead of hanging)."""
+    so ranks that wait for a missing peer fail instead of hanging). `device`
+    (a torch.device, for NCCL) binds the group to this rank's GPU."""
     if info.world <= 1:
         return None
     import torch.distributed as dist
-    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    kw = {} if device is None else {"device_id": device}
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
     return dist
 
 
