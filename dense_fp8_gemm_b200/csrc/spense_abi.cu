@@ -160,6 +160,10 @@ int l2_prefetch_knob() {
   static const int v = env_int("SPENSE_L2_PREFETCH", -1, -1, 1 << 20);
   return v;
 }
+// L2 prefetch depth of a planned launch (see l2_prefetch_knob).
+int l2_prefetch_for(const GemmPlan& pl) {
+  return l2_prefetch_knob() >= 0 ? l2_prefetch_knob() : (pl.cluster > 1 ? 4 : 0);
+}
 // Tokens per token tile (multiple of 16, at most 256); 0 (default) =
 // automatic (see make_plan).
 int token_tile_knob() {
@@ -498,7 +502,7 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
   p.producers = pl.producers;
   p.cluster = pl.cluster;
   p.recv_bytes = pl.recv_bytes;
-  p.l2_prefetch = l2_prefetch_knob() >= 0 ? l2_prefetch_knob() : (pl.cluster > 1 ? 4 : 0);
+  p.l2_prefetch = l2_prefetch_for(pl);
   p.x_warp = x_warp();
   // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
   // the workspace, which nothing sets, so every launch ends by timeout.
@@ -757,6 +761,59 @@ size_t spense_gemm_grouped_workspace_size(const spense_packed* const* Wps, int c
   GemmPlan pl;
   if (make_plan(Wps, count, M, info.sms, &pl) != SPENSE_OK) return 0;
   return pl.ws.total_device;
+}
+
+static_assert(SPENSE_PLAN_MAX_GRID == kMaxGrid, "plan introspection array size");
+
+spense_status spense_plan_shapes(int count, const int64_t* N, const int64_t* K, const int64_t* Kd, int64_t M,
+                                 int sms, spense_plan_info* out) {
+  if (out == nullptr || N == nullptr || K == nullptr || Kd == nullptr)
+    return fail(SPENSE_ERR_ARG, "out, N, K or Kd is NULL");
+  if (count < 1 || count > kMaxGroup)
+    return fail(SPENSE_ERR_ARG, "a launch takes 1 to %d packed weights, got %d", kMaxGroup, count);
+  if (sms < 1 || sms > 1024) return fail(SPENSE_ERR_ARG, "sms = %d outside [1, 1024]", sms);
+  std::vector<spense_packed> hs(static_cast<size_t>(count));
+  std::vector<const spense_packed*> ptrs(static_cast<size_t>(count));
+  for (int i = 0; i < count; ++i) {
+    if (N[i] < 1 || N[i] > (1 << 20)) return fail(SPENSE_ERR_SHAPE, "N = %lld outside [1, 2^20]", (long long)N[i]);
+    if (K[i] < 16 || K[i] > (1 << 20) || K[i] % 16 != 0)
+      return fail(SPENSE_ERR_SHAPE, "K = %lld must be a multiple of 16 in [16, 2^20]", (long long)K[i]);
+    if (Kd[i] < 0 || Kd[i] > K[i] || Kd[i] % 16 != 0)
+      return fail(SPENSE_ERR_SHAPE, "Kd = %lld must be a multiple of 16 in [0, K]", (long long)Kd[i]);
+    spense_packed& h = hs[static_cast<size_t>(i)];
+    h.device = 0;
+    h.N = N[i];
+    h.K = K[i];
+    h.Kd = Kd[i];
+    h.Ks = K[i] - Kd[i];
+    h.n_tiles = static_cast<int>((N[i] + kTileRows - 1) / kTileRows);
+    h.nsb = static_cast<int>((h.Ks + kSparseBlockCols - 1) / kSparseBlockCols);
+    h.ndb = static_cast<int>((Kd[i] + kDenseBlockCols - 1) / kDenseBlockCols);
+    ptrs[static_cast<size_t>(i)] = &h;
+  }
+  GemmPlan pl{};
+  const spense_status st = make_plan(ptrs.data(), count, M, sms, &pl);
+  if (st != SPENSE_OK) return st;
+  *out = spense_plan_info{};
+  out->npad = pl.npad;
+  out->box_rows = pl.box_rows;
+  out->m_tiles = pl.m_tiles;
+  out->n_tiles = pl.n_tiles;
+  out->tiles = pl.tiles;
+  out->ctas_per_sm = pl.ctas_per_sm;
+  out->cluster = pl.cluster;
+  out->grid = pl.grid;
+  out->stages = pl.stages;
+  out->nacc = pl.nacc;
+  out->tmem_cols = pl.tmem_cols;
+  out->smem_bytes = pl.smem_bytes;
+  out->stage_bytes = pl.stage_bytes;
+  out->recv_bytes = pl.recv_bytes;
+  out->l2_prefetch = l2_prefetch_for(pl);
+  out->total_blocks = pl.cta_start[pl.grid];
+  out->workspace_bytes = pl.ws.total_device;
+  for (int g = 0; g <= pl.grid; ++g) out->cta_start[g] = pl.cta_start[g];
+  return ok();
 }
 
 size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M) {

@@ -30,7 +30,7 @@ SYMBOLS = (
     "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
     "spense_gemm_grouped", "spense_gemm_grouped_workspace_size", "spense_gemm_grouped_ex",
     "spense_quantize", "spense_score_glu", "spense_score_workspace_size", "spense_select_dense",
-    "spense_pack_rows",
+    "spense_pack_rows", "spense_plan_shapes",
 )
 GEMM_X_PACKED_ORDER = 1
 MAX_GROUP = 4
@@ -56,6 +56,17 @@ class PackedInfo(ctypes.Structure):
 _lib = None
 
 
+PLAN_MAX_GRID = 320
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("npad", "box_rows", "m_tiles", "n_tiles", "tiles", "ctas_per_sm",
+                                              "cluster", "grid", "stages", "nacc")] + \
+               [(n, ctypes.c_uint32) for n in ("tmem_cols", "smem_bytes", "stage_bytes", "recv_bytes")] + \
+               [("l2_prefetch", ctypes.c_int32), ("total_blocks", ctypes.c_int64),
+                ("workspace_bytes", ctypes.c_uint64), ("cta_start", ctypes.c_int32 * (PLAN_MAX_GRID + 1))]
+
+
 def lib() -> ctypes.CDLL:
     """Load libspense.so (built in-tree by dense_fp8_gemm_b200.build)."""
     global _lib
@@ -74,6 +85,7 @@ def lib() -> ctypes.CDLL:
     L.spense_gemm_host_workspace_size.restype = SZ
     L.spense_free.argtypes = [P]
     L.spense_get_info.argtypes = [P, ctypes.POINTER(PackedInfo)]
+    L.spense_plan_shapes.argtypes = [ctypes.c_int, P, P, P, I64, ctypes.c_int, ctypes.POINTER(PlanInfo)]
     L.spense_workspace_status.argtypes = [P, P, ctypes.POINTER(U32)]
     L.spense_gemm_noalloc.argtypes = [P, P, P, I64, P, P]
     L.spense_gemm_grouped.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ, P]
@@ -381,6 +393,22 @@ def workspace_status(workspace: torch.Tensor, stream=None) -> int:
     _check(lib().spense_workspace_status(_dev_ptr(workspace, torch.uint8, "workspace"), _stream(stream),
                                          ctypes.byref(out)), "spense_workspace_status")
     return int(out.value)
+
+
+def plan_shapes(shapes, M: int, sms: int = 148) -> dict:
+    """spense_plan_shapes: the launch plan of a grouped GEMM over weights of
+    the given (N, K, Kd) shapes for M tokens on a device with `sms` SMs, from
+    the shapes alone (no GPU). Returns the plan's fields; cta_start as a list
+    of grid + 1 block indices."""
+    n = len(shapes)
+    arr = [np.ascontiguousarray([int(s[i]) for s in shapes], dtype=np.int64) for i in range(3)]
+    info = PlanInfo()
+    code = lib().spense_plan_shapes(n, *(a.ctypes.data_as(ctypes.c_void_p) for a in arr), int(M), int(sms),
+                                    ctypes.byref(info))
+    _check(code, "spense_plan_shapes")
+    out = {name: getattr(info, name) for name, _ in PlanInfo._fields_ if name != "cta_start"}
+    out["cta_start"] = list(info.cta_start[:info.grid + 1])
+    return out
 
 
 def version() -> str:

@@ -340,6 +340,41 @@ typedef struct spense_packed_info {
 
 SPENSE_API spense_status spense_get_info(const spense_packed* Wp, spense_packed_info* info);
 
+/* The launch plan a grouped GEMM would get, from shapes alone (no device
+ * memory, no GPU needed; for inspection and host-side tests of the planner).
+ * Member i is an N[i] x K[i] weight with Kd[i] dense columns (tail), all
+ * sharing one activation tensor of M tokens, planned for a device with `sms`
+ * SMs. Shape rules and errors are those of spense_pack and
+ * spense_gemm_grouped (members must share K). Blocks are numbered member by
+ * member, row tile by row tile (token tiles of one row tile consecutive),
+ * 2:4 blocks before dense blocks within a tile; CTA g of the launch streams
+ * blocks [cta_start[g], cta_start[g + 1]). With cluster > 1 the CTAs of one
+ * cluster (cluster consecutive CTAs) split the blocks of one tile. */
+#define SPENSE_PLAN_MAX_GRID 320
+typedef struct spense_plan_info {
+  int32_t npad;          /* tokens per token tile, padded to a multiple of 16 (the MMA N) */
+  int32_t box_rows;      /* activation rows one tile load covers */
+  int32_t m_tiles;       /* token tiles */
+  int32_t n_tiles;       /* 128-row weight tiles over all members */
+  int32_t tiles;         /* n_tiles * m_tiles */
+  int32_t ctas_per_sm;   /* 1 or 2 */
+  int32_t cluster;       /* 1 (stream-K) or the cluster size S splitting each tile's K */
+  int32_t grid;          /* CTAs */
+  int32_t stages;        /* shared-memory ring stages per CTA */
+  int32_t nacc;          /* accumulator buffers in tensor memory */
+  uint32_t tmem_cols;    /* tensor-memory columns allocated per CTA */
+  uint32_t smem_bytes;   /* dynamic shared memory per CTA */
+  uint32_t stage_bytes;  /* bytes of one ring stage */
+  uint32_t recv_bytes;   /* cluster mode: rank 0's area for the peers' partials */
+  int32_t l2_prefetch;   /* weight blocks per CTA prefetched into L2 at start */
+  int64_t total_blocks;  /* blocks the launch streams */
+  uint64_t workspace_bytes;                    /* spense_gemm_grouped_workspace_size */
+  int32_t cta_start[SPENSE_PLAN_MAX_GRID + 1]; /* [grid] = total_blocks */
+} spense_plan_info;
+
+SPENSE_API spense_status spense_plan_shapes(int count, const int64_t* N, const int64_t* K, const int64_t* Kd,
+                                            int64_t M, int sms, spense_plan_info* out);
+
 /* Reads and clears the status word a workspace carries. *status_out receives 0
  * when every kernel that used the workspace completed normally, else a bitwise
  * OR of SPENSE_DEVICE_* codes. Synchronizes `stream`. */
