@@ -261,8 +261,6 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // than one maximal block, so no CTA owns an empty range): small matrices are
   // split across fewer CTAs, which keeps the number of partials per tile low.
   long long grid = pl.total_cost / std::max<long long>(kCostSparse, min_cta_weight());
-  // Two CTAs per SM (two independent copy streams) when the token tile fits
-  // in half the shared and tensor memory; otherwise one.
   pl.bulk_split = bulk_split();
   pl.producers = producers();
   pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.any_sparse ? 256u : 128u);
