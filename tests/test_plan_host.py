@@ -1,5 +1,5 @@
 """Host-side checks of the launch planner (spense_plan_shapes, no GPU): for
-the workloads' shapes and token counts from 1 to 4096, every plan streams
+the workloads' shapes and token counts from 1 to 65535, every plan streams
 every weight block exactly once, keeps a cluster inside one tile, fits the
 shared-memory and tensor-memory budgets of its CTAs-per-SM choice, covers
 every token, and sizes its workspace for its partials; and the token-tile and
@@ -30,7 +30,7 @@ SHAPES = {
     "split": [(19200, 5120, 0), (6400, 5120, 5120)],           # output-split: 2:4 rows, dense rows
     "ragged": [(1000, 1024, 256), (136, 1024, 256)],
 }
-TOKENS = (1, 5, 8, 16, 32, 33, 64, 65, 128, 200, 256, 600, 4096)
+TOKENS = (1, 5, 8, 16, 32, 33, 64, 65, 128, 200, 256, 600, 4096, 65535)
 
 
 def blocks_of(N, K, Kd):
