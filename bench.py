@@ -1,16 +1,19 @@
 #!/usr/bin/env python
 """Benchmark of the Spense hybrid 2:4-sparse + dense FP8 GEMM on B200.
 
-Workload (default): the attention projections of a 32B-class decoder (hidden
-5120): q_proj 8192x5120, k_proj and v_proj 1024x5120, o_proj 5120x8192, FP8
-e4m3 weights with the last 25% of the input columns dense, M = 16 decode
-tokens. One step = the four GEMMs of one layer. Eight layers' packed weights
-(542 MB, more than the 126 MB L2) are rotated so every step streams its
-weights from HBM. Inputs are seeded synthetic tensors (no model weights).
+Workload (default): one decode step of a 36B-class decoder's projections
+(hidden 5120): per layer q/k/v (10240, 1024, 1024 x 5120, one grouped launch),
+o_proj 5120x10240, fused gate+up 55296x5120 and down 5120x27648, 64 distinct
+layers (24.8 GB of Spense weights, 34.6 GB as dense FP8), FP8 e4m3 weights
+with the last 25% of the input columns dense, M = 16 decode tokens; the same
+step at the other token counts of the workload (1, 4, 64, 256) is reported
+beside it. One step = every GEMM of every layer once, captured in one CUDA
+graph. Inputs are seeded synthetic tensors (no model weights); the weights
+are drawn on the GPU.
 
 Metric: weight-stream GB/s = algorithmic bytes (packed values + 2-bit
 metadata + dense columns + scales + activations + bf16 output) / time; also
-the speedup over the same kernel on the dense FP8 matrix (dense_frac = 1).
+the speedup over the same kernel on the dense FP8 matrices (dense_frac = 1).
 
 Prints one JSON line (rank 0). Multi-GPU runs are independent replicas (the
 GEMM has no exchange step), launched one process per GPU.
@@ -36,58 +39,101 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["spense", "reference"], default="spense")
-    ap.add_argument("--tokens", type=int, default=16, help="decode tokens M")
-    ap.add_argument("--layers", type=int, default=8, help="weight sets rotated between steps")
+    ap.add_argument("--workload", choices=sorted(STACKS), default="chain36b",
+                    help="chain36b: a 36B-class decoder's projections, 64 distinct layers (the headline); "
+                         "attn32b: a 32B-class decoder's attention projections, 8 distinct layers")
+    ap.add_argument("--tokens", type=int, default=16, help="decode tokens M of the headline line")
+    ap.add_argument("--layers", type=int, default=0, help="distinct layers in one step (0: the workload's)")
+    ap.add_argument("--sweep", default=None,
+                    help="comma-separated extra token counts timed on the same weights (default: the "
+                         "workload's other batch sizes; empty: none)")
     ap.add_argument("--dense-frac", type=float, default=0.25)
-    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline budget")
+    ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--op", choices=["gemm", "quantize", "score", "glu"], default="gemm",
-                    help="gemm: the hybrid GEMM (default, the headline); quantize: the per-token FP8 "
-                         "quantisation with the SpenseGPT+ column order fused in; score: the SpenseGPT+ "
-                         "dense-set scorer and top-Kd selection; glu: a 32B-class GLU MLP's three projections "
-                         "under the pages' GLU policy (gate/up output-split, down input-split, permutation folded)")
+                    help="gemm: the hybrid GEMM over a decoder stack (default, the headline); quantize: the "
+                         "per-token FP8 quantisation with the SpenseGPT+ column order fused in; score: the "
+                         "SpenseGPT+ dense-set scorer and top-Kd selection; glu: a 32B-class GLU MLP's three "
+                         "projections under the pages' GLU policy (gate/up output-split, down input-split, "
+                         "permutation folded)")
     return ap.parse_args()
 
 
-SHAPES = (("q_proj", 8192, 5120), ("k_proj", 1024, 5120), ("v_proj", 1024, 5120), ("o_proj", 5120, 8192))
-# One step = one layer's attention projections: q, k and v read the same hidden
-# state and run as one grouped launch; o_proj reads the attention output.
-GROUPS = ((0, 1, 2), (3,))
-
+# Decoder stacks the GEMM is measured on. One step = every GEMM of every layer
+# once (a decode step of the stack), the layers' weights all distinct, so each
+# step streams them from HBM. Launch groups: q, k and v read the same hidden
+# state and run as one grouped launch; each other projection is one launch.
+STACKS = {
+    "chain36b": {"workload": "CHAIN36B", "groups": ((0, 1, 2), (3,), (4,), (5,)),
+                 "names": ("qkv_grouped", "o_proj", "gate_up", "down")},
+    "attn32b": {"workload": "ATTN32B", "groups": ((0, 1, 2), (3,)), "layers": 8,
+                "names": ("qkv_grouped", "o_proj")},
+}
 
 L2_BYTES = 126 << 20
 
 
-def l2_note(sets, total):
-    rel = "larger" if total > L2_BYTES else "NOT larger"
-    return f"{sets} weight sets rotated per step ({total / 1e6:.0f} MB, {rel} than the 126 MB L2)"
+def stack_of(args):
+    from dense_fp8_gemm_b200 import workloads
+    st = STACKS[args.workload]
+    wl = getattr(workloads, st["workload"])
+    layers = args.layers or st.get("layers", wl.layers)
+    return wl, st["groups"], st["names"], layers
+
+
+def sweep_tokens(args):
+    wl, _, _, _ = stack_of(args)
+    if args.sweep is None:
+        return [m for m in wl.batches if m != args.tokens]
+    return [int(v) for v in args.sweep.split(",") if v.strip()]
+
+
+def group_members(wl, grp, dense_frac, dense=False):
+    from dense_fp8_gemm_b200 import workloads
+    return [(wl.shapes[i][1], wl.shapes[i][2],
+             wl.shapes[i][2] if dense else workloads.dense_count(wl.shapes[i][2], dense_frac)) for i in grp]
+
+
+def layer_bytes(wl, groups, M, dense_frac, dense=False):
+    """Algorithmic bytes of one layer's launches at M tokens."""
+    from dense_fp8_gemm_b200 import workloads
+    return sum(workloads.group_algorithmic_bytes(group_members(wl, g, dense_frac, dense), M) for g in groups)
+
+
+def step_bytes(args, M=None, dense=False):
+    wl, groups, _, layers = stack_of(args)
+    return layers * layer_bytes(wl, groups, args.tokens if M is None else M, args.dense_frac, dense)
+
+
+def step_flops(args, M=None):
+    from dense_fp8_gemm_b200 import workloads
+    wl, groups, _, layers = stack_of(args)
+    M = args.tokens if M is None else M
+    return layers * sum(workloads.useful_flops(n, k, kd, M) for g in groups
+                        for n, k, kd in group_members(wl, g, args.dense_frac))
 
 
 def workload_config(args):
+    wl, groups, names, layers = stack_of(args)
+    total = step_bytes(args)
     return {
-        "workload": f"attn32b q/k/v/o projections, decode M={args.tokens}",
-        "shapes": [f"{n}x{k}" for _, n, k in SHAPES],
-        "launches_per_step": "q+k+v grouped (shared input), o_proj",
+        "workload": f"{args.workload}: {layers} distinct decoder layers x {len(groups)} launches, decode "
+                    f"M={args.tokens}",
+        "shapes": [f"{label} {n}x{k}" for label, n, k in wl.shapes],
+        "launches_per_layer": list(names),
+        "layers": layers,
         "tokens": args.tokens,
         "dense_frac": args.dense_frac,
         "dense_columns": "tail (SpenseGPT)",
-        "weights": "FP8 e4m3 N(0,0.02) per-channel absmax scales; X N(0,1) per-token scales; seed 1",
-        "l2": l2_note(args.layers, args.layers * step_bytes(args)),
-        "graph": f"one CUDA graph per {args.layers} steps (the rotated layers back to back)",
+        "weights": f"FP8 e4m3 N(0,{wl.w_std}) per-channel absmax scales, drawn on the GPU (torch Philox, "
+                   f"seed {wl.seed}); X N(0,{wl.x_std}) per-token absmax scales",
+        "l2": f"inputs larger than L2: one step streams {total / 1e9:.2f} GB of distinct weights "
+              f"(L2 126 MB), no flush needed",
+        "graph": f"one CUDA graph per step ({layers * len(groups)} launches, programmatic dependent launch)",
     }
-
-
-def step_bytes(args, dense=False):
-    from dense_fp8_gemm_b200 import workloads
-    total = 0
-    for grp in GROUPS:
-        mem = [(SHAPES[i][1], SHAPES[i][2],
-                SHAPES[i][2] if dense else workloads.dense_count(SHAPES[i][2], args.dense_frac)) for i in grp]
-        total += workloads.group_algorithmic_bytes(mem, args.tokens)
-    return total
 
 
 KERNEL_SOURCES = ("gemm_sm100.cu", "sm100_ptx.cuh", "spense_internal.h")
@@ -103,12 +149,16 @@ def kernel_source_sha256():
     return h.hexdigest()
 
 
-def read_traffic():
-    """DRAM bytes per launch of spense_gemm_kernel from the committed ncu summary,
-    or None when the kernel sources have changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "spense_gemm_attn32b_m16_traffic.txt")
+def traffic_path(args):
+    return os.path.join(ROOT, "profiles", f"spense_gemm_{args.workload}_m{args.tokens}_traffic.txt")
+
+
+def read_traffic(args):
+    """DRAM bytes per launch of spense_gemm_kernel from the committed ncu record
+    of this workload, or None when there is none or the kernel sources have
+    changed since the counters were taken."""
     try:
-        with open(path) as f:
+        with open(traffic_path(args)) as f:
             rec = json.load(f)
         return rec["dram_bytes_per_launch_avg"] if rec["kernel_source_sha256"] == kernel_source_sha256() else None
     except Exception:
@@ -196,72 +246,142 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- CPU oracle timing
 
 
-def oracle_items(args, rows_per_shape: int):
-    """The bounded sample the CPU oracle runs: `rows_per_shape` output rows of
-    each projection, with the step's activations (q/k/v share one input)."""
+def host_cores():
+    """(nproc: CPUs this process may run on, std::thread::hardware_concurrency)."""
+    import oracle
+    try:
+        nproc = len(os.sched_getaffinity(0))
+    except Exception:
+        nproc = os.cpu_count() or 1
+    return nproc, oracle.hardware_concurrency()
+
+
+def group_inputs_host(args, M):
+    """Host activations of each launch group: X [M, K] e4m3 and s_x [M]."""
+    from dense_fp8_gemm_b200 import workloads
+    wl, groups, _, _ = stack_of(args)
+    return [workloads.make_activations(wl, g[0], M) for g in groups]
+
+
+def sample_items(args, layer, rows):
+    """Oracle work items of layer `layer`: for every weight, `rows` rows drawn
+    with its shape's columns and distribution (host generator, a stream of
+    their own) and the oracle's own keep mask. Item = (X, s_x, W, s_w, keep,
+    full N)."""
     import oracle
     from dense_fp8_gemm_b200 import workloads
-    wl = workloads.ATTN32B
-    acts = {0: workloads.make_activations(wl, 0, args.tokens), 3: workloads.make_activations(wl, 3, args.tokens)}
-    items, members = [], []
-    for grp in GROUPS:
-        X, s_x = acts[grp[0]]
-        mem = []
-        for i in grp:
-            w = workloads.make_weight(wl, i, args.dense_frac)
-            rows = np.linspace(0, w.N - 1, rows_per_shape).astype(np.int64)
-            keep = oracle.pack(w.W[rows], Kd=w.Kd)["keep"]
-            items.append((X, s_x, w.W[rows].copy(), w.s_w[rows].copy(), keep))
-            mem.append((rows_per_shape, w.K, w.Kd))
-        members.append(mem)
-    byts = sum(workloads.group_algorithmic_bytes(m, args.tokens) for m in members)
-    return items, byts
+    wl, groups, _, _ = stack_of(args)
+    acts = group_inputs_host(args, args.tokens)
+    items = []
+    for gi, g in enumerate(groups):
+        X, s_x = acts[gi]
+        for i in g:
+            w = workloads.make_weight(wl, i, args.dense_frac, layer=layer, rows=rows)
+            items.append((X, s_x, w.W, w.s_w, oracle.pack(w.W, Kd=w.Kd)["keep"], wl.shapes[i][1]))
+    return items
 
 
-def oracle_pass(items, nthreads):
+def full_layer_items(args, layer, dev):
+    """Oracle work items holding layer `layer`'s full weights: the same seeded
+    tensors the GPU arm packs (drawn on the GPU by the input generator, copied
+    to the host), with the oracle's own keep masks."""
     import oracle
-    for X, s_x, W, s_w, keep in items:
+    from dense_fp8_gemm_b200 import synth, workloads
+    wl, groups, _, _ = stack_of(args)
+    acts = group_inputs_host(args, args.tokens)
+    items = []
+    for gi, g in enumerate(groups):
+        X, s_x = acts[gi]
+        for i in g:
+            _, N, K = wl.shapes[i]
+            q, sc = synth.device_fp8_rows(wl.seed, workloads.weight_id(i, layer), (N, K), wl.w_std, dev)
+            W, s_w = q.cpu().numpy(), sc.cpu().numpy()
+            del q, sc
+            keep = oracle.pack(W, Kd=workloads.dense_count(K, args.dense_frac))["keep"]
+            items.append((X, s_x, W, s_w, keep, N))
+    return items
+
+
+def oracle_time(items, nthreads):
+    """Seconds the oracle takes over the items, each scaled from its rows to
+    its weight's full row count (1 for full weights)."""
+    import oracle
+    total = 0.0
+    for X, s_x, W, s_w, keep, n_full in items:
+        t0 = time.perf_counter()
         oracle.gemm(X, s_x, W, s_w, keep=keep, nthreads=nthreads)
+        total += (time.perf_counter() - t0) * n_full / W.shape[0]
+    return total
 
 
-def oracle_sample_rate(args, rows_per_shape: int, budget_s: float, nthreads: int):
-    """Times the CPU oracle (as it stands) on the bounded sample, repeating until
-    `budget_s` elapses. Returns (GB/s, seconds, passes)."""
-    items, byts = oracle_items(args, rows_per_shape)
-    reps, t0 = 0, time.perf_counter()
-    while True:
-        oracle_pass(items, nthreads)
-        reps += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
-    return byts * reps / el / 1e9, el, reps
+def cpu_baseline(args, dev):
+    """The CPU oracle (as it stands) on this step's workload, reported beside
+    the GPU number: single-threaded and on all host cores, median of 3 runs.
+    All cores: the full weights of the first and last layer, `rows` sampled
+    rows of every weight of the layers between (scaled by N / rows). One thread:
+    sampled rows of the first and last layer, scaled to the whole stack."""
+    wl, groups, _, layers = stack_of(args)
+    nproc, hwc = host_cores()
+    rows = 64
+    per_step = step_bytes(args)
+    t_setup = time.perf_counter()
+    ends = sorted({0, layers - 1})
+    full = {L: full_layer_items(args, L, dev) for L in ends}
+    mid = [sample_items(args, L, rows) for L in range(1, layers - 1)]
+    ends_sampled = [sample_items(args, L, rows) for L in ends]
+    setup_s = time.perf_counter() - t_setup
+    all_core, one = [], []
+    for _ in range(3):
+        all_core.append(sum(oracle_time(full[L], nproc) for L in ends) + sum(oracle_time(it, nproc) for it in mid))
+        one.append(sum(oracle_time(it, 1) for it in ends_sampled) * layers / len(ends))
+    t_all, t_one = statistics.median(all_core), statistics.median(one)
+    return {
+        "value": per_step / t_all / 1e9, "unit": "GB/s", "cores": nproc, "kind": "oracle",
+        "sample": (f"one decode step of {layers} layers at M={args.tokens}: full weights of layers {ends}, "
+                   f"{rows} sampled rows of every weight of the other layers scaled by N/{rows} "
+                   f"(extrapolated), all {nproc} cores, median of 3"),
+        "extrapolated": True,
+        "seconds_per_step": t_all,
+        "single_thread": {"value": per_step / t_one / 1e9, "unit": "GB/s", "cores": 1,
+                          "seconds_per_step": t_one,
+                          "sample": f"{rows} sampled rows of every weight of layers {ends}, scaled to all "
+                                    f"{layers} layers and full N (extrapolated), median of 3"},
+        "nproc": nproc, "hardware_concurrency": hwc, "setup_s": setup_s,
+    }
 
 
 # ----------------------------------------------------------------------------- reference arm
 
 
 def run_reference(args):
+    """The CPU oracle timed as the reference arm, on a bounded sample of this
+    workload per step: `rows` rows of every weight of one layer (the layers
+    rotate), all host cores. The line's value scales the sample to the full
+    step's algorithmic bytes."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cores = os.cpu_count() or 1
-    rows = 32  # bounded sample per step: 32 output rows of each projection
-    items, per_step = oracle_items(args, rows)
-    for _ in range(args.warmup):
-        oracle_pass(items, cores)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_pass(items, cores)
-    el = time.perf_counter() - t0
-    value = per_step * args.steps / el / 1e9
-    sample = f"{rows} output rows of each of q/k/v/o per step (M={args.tokens}), all {cores} host threads"
+    wl, groups, _, layers = stack_of(args)
+    nproc, hwc = host_cores()
+    rows = 128
+    pool = [sample_items(args, L, rows) for L in sorted({0, layers // 2, layers - 1})]
+    for i in range(args.warmup):
+        oracle_time(pool[i % len(pool)], nproc)
+    t_sample = 0.0
+    for i in range(args.steps):
+        t_sample += oracle_time(pool[i % len(pool)], nproc)  # each layer scaled to full N
+    per_layer_s = t_sample / max(1, args.steps)
+    step_s = per_layer_s * layers
+    value = step_bytes(args) / step_s / 1e9
+    sample = (f"{rows} sampled rows of every weight of one layer per step (M={args.tokens}), scaled to full N "
+              f"and {layers} layers (extrapolated), all {nproc} host threads")
     line = {
         "impl": "reference", "metric": "spense_fp8_weight_stream_GBps", "value": value, "unit": "GB/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": el / max(1, args.steps) * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": workload_config(args),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": nproc, "kind": "oracle", "sample": sample,
+                         "hardware_concurrency": hwc},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -274,7 +394,7 @@ def run_reference(args):
 def run_spense(args):
     import torch
 
-    from dense_fp8_gemm_b200 import replicas, spense, workloads
+    from dense_fp8_gemm_b200 import replicas, spense, synth, workloads
 
     ranks = replicas.from_env()
     world, rank, local = ranks.world, ranks.rank, ranks.local
@@ -282,171 +402,158 @@ def run_spense(args):
     dev = torch.device("cuda", local)
     replicas.init(ranks, "nccl", device=dev)
 
-    M = args.tokens
-    wl = workloads.ATTN32B
-    # ---- weights: one synthetic layer, packed into `layers` distinct buffer sets
-    host_w = [workloads.make_weight(wl, i, args.dense_frac) for i in range(len(SHAPES))]
-    layers_sp, layers_dn = [], []
-    for _ in range(args.layers):
+    wl, groups, names, layers = stack_of(args)
+    M0 = args.tokens
+    Ms = [M0] + [m for m in sweep_tokens(args) if m != M0]
+    Mmax = max(Ms)
+
+    # ---- weights: every layer distinct, drawn on the GPU, packed twice: the
+    # Spense format (dense_frac of the columns dense, the rest 2:4) and all
+    # dense (the same kernel on the dense FP8 matrix, Kd = K).
+    t_gen = time.perf_counter()
+    arms = {"spense": [], "dense": []}
+    for L in range(layers):
         sp, dn = [], []
-        for w in host_w:
-            Wd = torch.from_numpy(w.W).to(dev)
-            sd = torch.from_numpy(w.s_w).to(dev)
-            sp.append(spense.pack(Wd, sd, Kd=w.Kd))
-            dn.append(spense.pack(Wd, sd, Kd=w.K))
-            del Wd
-        layers_sp.append(sp)
-        layers_dn.append(dn)
-    # activations: q/k/v share the hidden state, o_proj reads the attention output
-    host_x = {grp[0]: workloads.make_activations(wl, grp[0], M) for grp in GROUPS}
-    dev_x = {k: (torch.from_numpy(v[0]).to(dev), torch.from_numpy(v[1]).to(dev)) for k, v in host_x.items()}
-    Ys = [torch.empty((M, n), dtype=torch.bfloat16, device=dev) for _, n, _ in SHAPES]
-    ws_bytes = max(spense.grouped_workspace_size([L[i] for i in grp], M)
-                   for L in (layers_sp[0], layers_dn[0]) for grp in GROUPS)
-    ws = spense.new_workspace(ws_bytes, dev)
+        for i, (_, N, K) in enumerate(wl.shapes):
+            q, sc = synth.device_fp8_rows(wl.seed, workloads.weight_id(i, L), (N, K), wl.w_std, dev)
+            sp.append(spense.pack(q, sc, Kd=workloads.dense_count(K, args.dense_frac)))
+            dn.append(spense.pack(q, sc, Kd=K))
+            del q, sc
+        arms["spense"].append(sp)
+        arms["dense"].append(dn)
     torch.cuda.synchronize()
+    gen_s = time.perf_counter() - t_gen
 
-    def launch_layer(packs, stream, events=None):
-        for gi, grp in enumerate(GROUPS):
-            X, sx = dev_x[grp[0]]
-            if events is not None:
-                events[gi][0].record(stream)
-            spense.gemm_grouped([packs[i] for i in grp], X, sx, [Ys[i] for i in grp], ws, stream)
-            if events is not None:
-                events[gi][1].record(stream)
+    # ---- activations (one per launch group, Mmax rows; M-token calls use the
+    # first M rows) and outputs (one per weight, reused by every layer)
+    acts = group_inputs_host(args, Mmax)
+    X = [torch.from_numpy(x).to(dev) for x, _ in acts]
+    SX = [torch.from_numpy(sx).to(dev) for _, sx in acts]
+    Y = [[torch.empty((Mmax, wl.shapes[i][1]), dtype=torch.bfloat16, device=dev) for i in g] for g in groups]
+    ws_bytes = max(spense.grouped_host_workspace_size([arms[a][0][i] for i in g], m)
+                   for a in arms for g in groups for m in Ms)
+    ws = spense.new_workspace(ws_bytes, dev)
+    stream = torch.cuda.current_stream()
 
-    def capture_chain(layer_list):
-        """One graph over all layers in sequence (a decode step of the whole stack)."""
-        for L in layer_list:
-            launch_layer(L, torch.cuda.current_stream())
+    def prepared(arm, M, gis=None):
+        """PreparedGrouped calls of one step (layer by layer) at M tokens."""
+        calls = []
+        for Lw in arms[arm]:
+            for gi, g in enumerate(groups):
+                if gis is not None and gi not in gis:
+                    continue
+                calls.append(spense.PreparedGrouped([Lw[i] for i in g], X[gi][:M], SX[gi][:M],
+                                                    [y[:M] for y in Y[gi]], ws))
+        return calls
+
+    def capture(calls):
+        """One CUDA graph of the calls in order; run once eagerly first (plans
+        and attributes are set up outside capture) and replayed once after
+        capture (graph upload), so no timed replay pays either."""
+        for c in calls:
+            c(stream)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            for L in layer_list:
-                launch_layer(L, torch.cuda.current_stream())
+        with torch.cuda.graph(g, stream=stream):
+            for c in calls:
+                c(stream)
+        g.replay()
         torch.cuda.synchronize()
         return g
 
-    def capture(layer_list, with_events=False):
-        graphs, evs = [], []
-        for L in layer_list:
-            launch_layer(L, torch.cuda.current_stream())  # warm (attribute setup outside capture)
-        torch.cuda.synchronize()
-        for L in layer_list:
-            g = torch.cuda.CUDAGraph()
-            e = [(torch.cuda.Event(enable_timing=True, external=True),
-                  torch.cuda.Event(enable_timing=True, external=True)) for _ in GROUPS] if with_events else None
-            with torch.cuda.graph(g):
-                launch_layer(L, torch.cuda.current_stream(), e)
-            graphs.append(g)
-            evs.append(e)
-        torch.cuda.synchronize()
-        return graphs, evs
-
-    def timed(graphs, chain, steps, warmup, clocks=None):
-        # Steps run as whole-stack graphs (all rotated layers back to back, so
-        # each launch overlaps the previous one's tail); a remainder of fewer
-        # than `layers` steps uses the per-layer graphs.
-        def run(n):
-            for _ in range(n // len(graphs)):
-                chain.replay()
-            for i in range(n % len(graphs)):
-                graphs[i].replay()
-        run(warmup)
+    def timed(g, steps, warmup, clocks=None):
+        for _ in range(warmup):
+            g.replay()
         torch.cuda.synchronize()
         replicas.barrier(ranks)
         torch.cuda.synchronize()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         w0 = time.time()
-        e0.record()
-        run(steps)
-        e1.record()
+        e0.record(stream)
+        for _ in range(steps):
+            g.replay()
+        e1.record(stream)
         torch.cuda.synchronize()
         if clocks is not None:
             clocks.mark(w0, time.time())
         replicas.barrier(ranks)
         return e0.elapsed_time(e1) / 1e3  # seconds
 
-    g_sp, _ = capture(layers_sp)
-    g_dn, _ = capture(layers_dn)
-    c_sp = capture_chain(layers_sp)
-    c_dn = capture_chain(layers_dn)
-
+    launches_per_step = layers * len(groups)
+    g_sp = capture(prepared("spense", M0))
+    g_dn = capture(prepared("dense", M0))
     with ClockSampler(local) as clocks:
-        t_sp = timed(g_sp, c_sp, args.steps, args.warmup, clocks)
-    t_dn = timed(g_dn, c_dn, args.steps, args.warmup)
-
+        t_sp = timed(g_sp, args.steps, args.warmup, clocks)
+    t_dn = timed(g_dn, args.steps, args.warmup)
+    del g_sp, g_dn
     t_sp, t_dn = replicas.max_over_ranks(ranks, [t_sp, t_dn], device=dev)
-
     per_step = step_bytes(args)
     value = replicas.job_rate(per_step * args.steps, world, t_sp) / 1e9
-    launches = args.steps * len(GROUPS)
-
-    # ---- dominant kernel: per-launch device time from events captured around each launch
-    g_ev, evs = capture(layers_sp, with_events=True)
-    dur = [[] for _ in GROUPS]
-    reps = max(8, min(args.steps, 64))
-    for i in range(reps):
-        g_ev[i % len(g_ev)].replay()
-        torch.cuda.synchronize()
-        for gi, (a, b) in enumerate(evs[i % len(g_ev)]):
-            dur[gi].append(a.elapsed_time(b) / 1e3)
-    per_launch = [statistics.median(d) for d in dur]  # isolated: event nodes serialize the launches
-    # The timed region holds only spense_gemm_kernel launches (tail dense set: no gather), so the
-    # average launch duration over it is t_sp / launches and the bytes per launch average the
-    # step's algorithmic bytes over its launches.
-    avg_launch_s = t_sp / launches
-    bytes_per_launch = per_step / len(GROUPS)
-    achieved = bytes_per_launch / avg_launch_s / 1e9
     peak, peak_kind = read_peaks()
-    del g_ev, evs
 
-    # ---- e2e: host buffers in, host buffers out, copies inside the timed region.
-    # Each group's X and x_scale sit in one pinned host buffer and one device
-    # buffer (one host-to-device copy per group); all outputs of a step sit in
-    # one device buffer (one device-to-host copy per step); the GEMM calls are
-    # prepared once per layer (their arguments marshalled once).
-    import torch as _t
-    in_host, in_dev, in_views = {}, {}, {}
-    for k, (xh, sxh) in host_x.items():
-        nx = xh.size
-        buf_h = _t.empty(nx + 4 * M, dtype=_t.uint8).pin_memory()
-        buf_h[:nx] = _t.from_numpy(xh.reshape(-1))
-        buf_h[nx:] = _t.from_numpy(sxh.view(np.uint8))
-        buf_d = _t.empty_like(buf_h, device=dev)
-        in_host[k], in_dev[k] = buf_h, buf_d
-        in_views[k] = (buf_d[:nx].view(M, -1), buf_d[nx:].view(_t.float32))
-    offs = np.cumsum([0] + [M * n for _, n, _ in SHAPES])
-    out_dev = _t.empty(int(offs[-1]), dtype=_t.bfloat16, device=dev)
-    out_host = _t.empty(int(offs[-1]), dtype=_t.bfloat16).pin_memory()
-    y_views = [out_dev[int(offs[i]):int(offs[i + 1])].view(M, SHAPES[i][1]) for i in range(len(SHAPES))]
-    calls = [[spense.PreparedGrouped([layer[i] for i in grp], in_views[grp[0]][0], in_views[grp[0]][1],
-                                     [y_views[i] for i in grp], ws) for grp in GROUPS] for layer in layers_sp]
-    stream = torch.cuda.current_stream()
+    # ---- per launch group: the group's launches of all layers back to back
+    sub_steps = max(3, args.steps // 4)
+    per_group = {}
+    for gi, name in enumerate(names):
+        res = {}
+        for arm in ("spense", "dense"):
+            g = capture(prepared(arm, M0, gis={gi}))
+            t = timed(g, sub_steps, 2)
+            del g
+            b = layers * workloads.group_algorithmic_bytes(group_members(wl, groups[gi], args.dense_frac,
+                                                                         arm == "dense"), M0)
+            res[arm] = (t / sub_steps / layers, b / layers)
+        us, byt = res["spense"]
+        per_group[name] = {"us_per_launch": us * 1e6, "GBps": byt / us / 1e9, "frac": byt / us / 1e9 / peak,
+                           "dense_fp8_us": res["dense"][0] * 1e6, "speedup_vs_dense_fp8": res["dense"][0] / us}
 
-    def e2e_step(layer_calls):
-        for grp, call in zip(GROUPS, layer_calls):
-            in_dev[grp[0]].copy_(in_host[grp[0]], non_blocking=True)
-            call(stream)
-        out_host.copy_(out_dev, non_blocking=True)
-        stream.synchronize()
+    # ---- other token counts on the same weights
+    per_m = {}
+    for M in Ms[1:]:
+        res = {}
+        for arm in ("spense", "dense"):
+            g = capture(prepared(arm, M))
+            res[arm] = timed(g, sub_steps, 2) / sub_steps
+            del g
+        b = step_bytes(args, M)
+        per_m[str(M)] = {"ms_per_step": res["spense"] * 1e3, "GBps": b / res["spense"] / 1e9,
+                         "frac": b / res["spense"] / 1e9 / peak, "tflops": step_flops(args, M) / res["spense"] / 1e12,
+                         "dense_fp8_ms_per_step": res["dense"] * 1e3,
+                         "speedup_vs_dense_fp8": res["dense"] / res["spense"]}
 
-    e2e_steps = max(4, min(args.steps, 200))
-    for i in range(min(args.warmup, 8)):
-        e2e_step(calls[i % args.layers])
-    replicas.barrier(ranks)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(e2e_steps):
-        e2e_step(calls[i % args.layers])
-    e1.record()
+    # ---- e2e: one decode step of the stack through the C ABI, eager: the
+    # first launch takes the hidden state from pinned host memory
+    # (spense_gemm_grouped_host with GEMM_HOST_X, copy inside the call), the
+    # last returns its output to pinned host memory (GEMM_HOST_Y: copy inside
+    # the call, which synchronizes), the launches between run on device
+    # buffers. The timed region holds every copy and the final synchronization.
+    x_host = torch.from_numpy(acts[0][0][:M0].copy()).pin_memory()
+    sx_host = torch.from_numpy(acts[0][1][:M0].copy()).pin_memory()
+    last_g = groups[-1]
+    y_host = [torch.empty((M0, wl.shapes[i][1]), dtype=torch.bfloat16).pin_memory() for i in last_g]
+    calls = prepared("spense", M0)
+    calls[0] = spense.PreparedGroupedHost([arms["spense"][0][i] for i in groups[0]], x_host, sx_host,
+                                          [y[:M0] for y in Y[0]], ws, spense.GEMM_HOST_X)
+    calls[-1] = spense.PreparedGroupedHost([arms["spense"][-1][i] for i in last_g], X[-1][:M0], SX[-1][:M0],
+                                           y_host, ws, spense.GEMM_HOST_Y)
+
+    def e2e_step():
+        for c in calls:
+            c(stream)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
     torch.cuda.synchronize()
-    t_e2e = replicas.max_over_ranks(ranks, [e0.elapsed_time(e1) / 1e3], device=dev)[0]
-    h2d = sum(M * SHAPES[g[0]][2] + 4 * M for g in GROUPS)
-    d2h = sum(2 * M * n for _, n, _ in SHAPES)
-    e2e_value = replicas.job_rate(per_step * e2e_steps, world, t_e2e) / 1e9
+    replicas.barrier(ranks)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    t_e2e = time.perf_counter() - t0
+    t_e2e = replicas.max_over_ranks(ranks, [t_e2e], device=dev)[0]
+    h2d = x_host.numel() + 4 * sx_host.numel()
+    d2h = sum(2 * y.numel() for y in y_host)
+    e2e_value = replicas.job_rate(per_step * args.steps, world, t_e2e) / 1e9
 
     status = spense.workspace_status(ws)
     if status != 0:
@@ -454,15 +561,12 @@ def run_spense(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cores = os.cpu_count() or 1
-        gbs, el, reps_c = oracle_sample_rate(args, 256, args.cpu_seconds, cores)
-        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": f"256 output rows of each of q/k/v/o, M={args.tokens}, {reps_c} passes in {el:.1f} s"}
+        cpu = cpu_baseline(args, dev)
 
     if rank == 0:
-        kd = [workloads.dense_count(k, args.dense_frac) for _, _, k in SHAPES]
-        tflops = sum(workloads.useful_flops(n, k, kd[i], M) for i, (_, n, k) in enumerate(SHAPES)) \
-            * args.steps * world / t_sp / 1e12
+        avg_launch_s = t_sp / (args.steps * launches_per_step)
+        bytes_per_launch = per_step / launches_per_step
+        achieved = bytes_per_launch / avg_launch_s / 1e9
         line = {
             "metric": "spense_fp8_weight_stream_GBps", "value": value, "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_sp / args.steps * 1e3,
@@ -470,23 +574,29 @@ def run_spense(args):
             "data": "synthetic", "config": workload_config(args),
             "speedup_vs_dense_fp8": t_dn / t_sp,
             "dense_fp8_GBps": step_bytes(args, dense=True) * args.steps * world / t_dn / 1e9,
-            "tflops": tflops,
+            "dense_fp8_ms_per_step": t_dn / args.steps * 1e3,
+            "tflops": step_flops(args) * args.steps * world / t_sp / 1e12,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": read_traffic(), "peak_source": peak_kind,
+                         "frac": achieved / peak, "traffic": read_traffic(args), "peak_source": peak_kind,
                          "kernel": "spense_gemm_kernel", "avg_launch_us": avg_launch_s * 1e6,
-                         "bytes_per_launch": bytes_per_launch,
-                         "isolated_launch_us": {"qkv_grouped": per_launch[0] * 1e6, "o_proj": per_launch[1] * 1e6}},
+                         "bytes_per_launch": bytes_per_launch, "launches_per_step": launches_per_step},
+            "per_launch_group": per_group,
+            "per_tokens": per_m,
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
+            "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": t_e2e / args.steps * 1e3,
+                    "path": "eager C-ABI calls; first spense_gemm_grouped_host(GEMM_HOST_X), last "
+                            "spense_gemm_grouped_host(GEMM_HOST_Y), host clock"},
+            "gpu_launches": args.steps * launches_per_step,
+            "setup_s": gen_s,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
 
-    for L in layers_sp + layers_dn:
-        for p in L:
-            p.free()
-    del g_sp, g_dn, c_sp, c_dn  # graphs are released before the process group goes away
+    for arm in arms.values():
+        for Lw in arm:
+            for pw in Lw:
+                pw.free()
     replicas.finalize(ranks)
     return 0
 
@@ -692,7 +802,6 @@ def run_glu(args):
     input-split layout (gate+up as one K-split matrix, down with a tail set)."""
     import torch
     from dense_fp8_gemm_b200 import spense, synth, workloads
-    import oracle
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     H, I, M = 5120, 25600, args.tokens
@@ -700,7 +809,7 @@ def run_glu(args):
     Ns = I - Nd
     layers = 2
     D = synth.scored_dense_idx(2, 5, I, Nd)
-    pi = oracle.glu_order(I, D)
+    pi = spense.glu_order(I, D)  # the library's GLU order: other indices ascending, then the dense set
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(dev)
     sets, base = [], []
     for L in range(layers):

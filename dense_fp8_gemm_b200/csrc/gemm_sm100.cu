@@ -307,9 +307,11 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   // blocks; with x_warp the next warp copies the activation tiles.
   const int x_loader = p.x_warp ? 5 + p.producers : -1;
   const uint32_t bar2_threads = 32u * static_cast<uint32_t>(p.producers + p.x_warp);
-  // Test of the failure path: every loader waits (bounded) on a word nothing
-  // sets, before any copy is issued, so the timeout leaves no transfer in flight.
+  // Test build only (SPENSE_TEST_HOOKS): to exercise the failure path, every
+  // loader waits (bounded) on a word nothing sets, before any copy is issued,
+  // so the timeout leaves no transfer in flight.
   auto test_gate_wait = [&]() {
+#ifdef SPENSE_TEST_HOOKS
     if (lane != 0 || p.test_gate == nullptr) return;
     const uint64_t t0 = ptx::globaltimer();
     while (*reinterpret_cast<const volatile unsigned int*>(p.test_gate) == 0u && !*abort_flag) {
@@ -320,6 +322,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       }
       __nanosleep(1000);
     }
+#endif
   };
 
   if (warp == x_loader) {

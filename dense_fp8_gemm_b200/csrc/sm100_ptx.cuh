@@ -220,12 +220,6 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
-// Arrive on an mbarrier of another CTA of the cluster, releasing this
-// thread's prior writes (and those ordered before it) at cluster scope.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
 // Arrive on an mbarrier of another CTA of the cluster without ordering any
 // memory access (a pure signal).
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
@@ -269,35 +263,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Asynchronous 16-byte store into another CTA's shared memory; on arrival it
-// performs complete_tx(16) on that CTA's mbarrier (both addresses from mapa).
-__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
-                                            uint32_t cluster_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   cluster_addr),
-               "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
-               : "memory");
-}
-
 // 16-byte global store.
 __device__ __forceinline__ void st_global_v4(void* ptr, uint4 v) {
   asm volatile("st.global.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
-__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t cluster_addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(cluster_addr)
-               : "memory");
-  return v;
-}
-
-// Store to another CTA's shared memory (address from mapa).
-__device__ __forceinline__ void st_dsmem_v4(uint32_t cluster_addr, float4 v) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(cluster_addr), "f"(v.x), "f"(v.y),
-               "f"(v.z), "f"(v.w)
                : "memory");
 }
 
@@ -314,11 +282,6 @@ __device__ __forceinline__ void st_smem_v4(uint32_t saddr, float4 v) {
                : "memory");
 }
 
-// Arrive on the cluster barrier without waiting (releases prior writes).
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-
 // Arrive on the cluster barrier without waiting and without ordering any
 // earlier memory access.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -328,21 +291,6 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 // Wait for the cluster barrier phase this thread arrived on (acquire).
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Per-thread form of cluster_wait (no warp convergence required).
-__device__ __forceinline__ void cluster_wait_thread() {
-  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
-}
-
-// Per-thread form of cluster_arrive_relaxed.
-__device__ __forceinline__ void cluster_arrive_thread_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
-}
-
-// Whole-cluster barrier (every thread of every CTA of the cluster).
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- descriptors

@@ -10,6 +10,7 @@
 #include <mutex>
 #include <new>
 #include <string>
+#include <unordered_map>
 #include <vector>
 
 #include <cudaTypedefs.h>
@@ -379,15 +380,14 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     }
   }
   pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes + pl.recv_bytes;
-  int64_t n_sum = 0;
-  for (int i = 0; i < count; ++i) n_sum += hs[i]->N;
   WorkspaceLayout& w = pl.ws;
   size_t off = 256;  // header: status word
   w.counters_off = off;
   w.counters_bytes = round_up(static_cast<size_t>(pl.tiles) * 4, 256);
   off += w.counters_bytes;
   w.partials_off = off;
-  w.partials_bytes = static_cast<size_t>(pl.grid) * 2 * pl.npad * kTileRows * 4;
+  // fp32 partials of shared tiles: stream-K only (a cluster reduces in shared memory)
+  w.partials_bytes = pl.cluster > 1 ? 0 : static_cast<size_t>(pl.grid) * 2 * pl.npad * kTileRows * 4;
   off += w.partials_bytes;
   w.xg_off = off;
   w.xg_bytes = h0->perm ? round_up(static_cast<size_t>(M * h0->K), 256) : 0;
@@ -398,7 +398,7 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   w.stage_sx_off = off;
   off += round_up(static_cast<size_t>(M) * 4, 256);
   w.stage_y_off = off;
-  off += round_up(static_cast<size_t>(M * n_sum) * 2, 256);
+  for (int i = 0; i < count; ++i) off += round_up(static_cast<size_t>(M * hs[i]->N) * 2, 256);
   w.total_host = off;
   *out = pl;
   return SPENSE_OK;
@@ -502,10 +502,14 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
   p.recv_bytes = pl.recv_bytes;
   p.l2_prefetch = l2_prefetch_for(pl);
   p.x_warp = x_warp();
-  // SPENSE_TEST_STALL=1 (tests only): the loaders wait on header word 16 of
-  // the workspace, which nothing sets, so every launch ends by timeout.
+#ifdef SPENSE_TEST_HOOKS
+  // Test build only: with SPENSE_TEST_STALL=1 the loaders wait on header word
+  // 16 of the workspace, which nothing sets, so every launch ends by timeout.
   static const bool stall = env_int("SPENSE_TEST_STALL", 0, 0, 1) == 1;
   p.test_gate = stall ? reinterpret_cast<const unsigned int*>(ws + 64) : nullptr;
+#else
+  p.test_gate = nullptr;
+#endif
   out->smem = pl.smem_bytes;
   return SPENSE_OK;
 }
@@ -531,9 +535,10 @@ spense_status run_gemm(const spense_packed* const* hs, int count, const uint8_t*
 }
 
 // Launch cache: repeated calls with the same weights, shapes, pointers and
-// workspace (a decode loop) reuse the plan, the parameter block and the
-// tensor map instead of building them again. Keyed by the handles' unique
-// ids, so a freed and reallocated handle never matches an old entry.
+// workspace (a decode loop, or the layers of a model issued one after
+// another) reuse the plan, the parameter block and the tensor map instead of
+// building them again. Keyed by the handles' unique ids, so a freed and
+// reallocated handle never matches an old entry.
 struct LaunchKey {
   int device = -1, count = 0;
   uint64_t ids[kMaxGroup] = {};
@@ -554,15 +559,116 @@ struct LaunchKey {
   }
 };
 
+struct LaunchKeyHash {
+  size_t operator()(const LaunchKey& k) const {
+    uint64_t h = 1469598103934665603ull;  // FNV-1a over the fields that identify a call
+    auto mix = [&h](uint64_t v) {
+      for (int b = 0; b < 8; ++b) {
+        h ^= (v >> (8 * b)) & 0xffu;
+        h *= 1099511628211ull;
+      }
+    };
+    mix(static_cast<uint64_t>(k.device));
+    mix(static_cast<uint64_t>(k.count));
+    mix(static_cast<uint64_t>(k.M));
+    mix(reinterpret_cast<uintptr_t>(k.X));
+    mix(reinterpret_cast<uintptr_t>(k.x_scale));
+    mix(reinterpret_cast<uintptr_t>(k.ws));
+    mix(k.flags);
+    for (int i = 0; i < k.count; ++i) {
+      mix(k.ids[i]);
+      mix(reinterpret_cast<uintptr_t>(k.Ys[i]));
+      mix(static_cast<uint64_t>(k.ldy[i]));
+    }
+    return static_cast<size_t>(h);
+  }
+};
+
 struct LaunchCacheEntry {
-  LaunchKey key;
   size_t ws_needed = 0;
   PreparedLaunch launch;
 };
 
-constexpr size_t kLaunchCacheSize = 32;
+// Room for the distinct launches of a whole decoder stack (64 layers x a few
+// GEMMs each, several token counts); when full it starts over.
+constexpr size_t kLaunchCacheSize = 4096;
 std::mutex g_launch_mu;
-std::vector<LaunchCacheEntry>* g_launch_cache = new std::vector<LaunchCacheEntry>();  // most recent first
+auto* g_launch_cache = new std::unordered_map<LaunchKey, LaunchCacheEntry, LaunchKeyHash>();
+
+// Plans (or finds in the cache) and enqueues one grouped launch; arguments
+// validated by the caller. Device pointers only.
+spense_status launch_grouped(const spense_packed* const* Wps, int count, const uint8_t* X, const float* x_scale,
+                             int64_t M, uint16_t* const* Ys, const int64_t* ldy, void* workspace,
+                             size_t workspace_bytes, unsigned int flags, int dev, const DeviceInfo& info,
+                             cudaStream_t stream) {
+  LaunchKey key;
+  key.device = dev;
+  key.count = count;
+  for (int i = 0; i < count; ++i) {
+    key.ids[i] = Wps[i]->id;
+    key.Ys[i] = Ys[i];
+    key.ldy[i] = ldy != nullptr ? ldy[i] : Wps[i]->N;
+  }
+  key.M = M;
+  key.X = X;
+  key.x_scale = x_scale;
+  key.ws = workspace;
+  key.flags = flags;
+  {
+    std::lock_guard<std::mutex> lk(g_launch_mu);
+    auto it = g_launch_cache->find(key);
+    if (it != g_launch_cache->end()) {
+      if (workspace_bytes < it->second.ws_needed)
+        return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                    it->second.ws_needed);
+      return enqueue_gemm(it->second.launch, stream);
+    }
+  }
+  GemmPlan pl;
+  spense_status st = make_plan(Wps, count, M, info.sms, &pl);
+  if (st != SPENSE_OK) return st;
+  if (workspace_bytes < pl.ws.total_device)
+    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
+                pl.ws.total_device);
+  LaunchCacheEntry entry;
+  entry.ws_needed = pl.ws.total_device;
+  st = prepare_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
+                    (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u, ldy, &entry.launch);
+  if (st != SPENSE_OK) return st;
+  st = enqueue_gemm(entry.launch, stream);
+  if (st != SPENSE_OK) return st;
+  {
+    std::lock_guard<std::mutex> lk(g_launch_mu);
+    if (g_launch_cache->size() >= kLaunchCacheSize) g_launch_cache->clear();
+    g_launch_cache->emplace(key, entry);
+  }
+  return SPENSE_OK;
+}
+
+// Validates the host-side order arguments shared by spense_pack and
+// spense_glu_order: dense_idx strictly ascending in [0, K).
+spense_status check_dense_idx(const int32_t* dense_idx, int64_t Kd, int64_t K) {
+  for (int64_t j = 0; j < Kd; ++j) {
+    if (dense_idx[j] < 0 || dense_idx[j] >= K)
+      return fail(SPENSE_ERR_DENSE_IDX, "dense_idx[%lld] = %d outside [0, %lld)", (long long)j, dense_idx[j],
+                  (long long)K);
+    if (j > 0 && dense_idx[j] <= dense_idx[j - 1])
+      return fail(SPENSE_ERR_DENSE_IDX, "dense_idx is not strictly ascending at %lld", (long long)j);
+  }
+  return SPENSE_OK;
+}
+
+// The packed column order of a dense set (Technical Summary §2.B: the dense
+// indices permuted into one contiguous block after the others): every index
+// not in dense_idx, ascending, then dense_idx. dense_idx validated.
+void dense_block_order(const int32_t* dense_idx, int64_t Kd, int64_t K, int32_t* order) {
+  std::vector<char> dense(static_cast<size_t>(K), 0);
+  for (int64_t j = 0; j < Kd; ++j) dense[static_cast<size_t>(dense_idx[j])] = 1;
+  int64_t o = 0;
+  for (int64_t k = 0; k < K; ++k)
+    if (!dense[static_cast<size_t>(k)]) order[o++] = static_cast<int32_t>(k);
+  for (int64_t j = 0; j < Kd; ++j) order[o++] = dense_idx[j];
+}
 
 // ---------------------------------------------------------------- allocation-free entry point
 // Scratch for spense_gemm_noalloc: a fixed array in device memory that every
@@ -571,18 +677,47 @@ std::vector<LaunchCacheEntry>* g_launch_cache = new std::vector<LaunchCacheEntry
 // cudaGetSymbolAddress, looked up once per device with that device current.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SPENSE_NOALLOC_SCRATCH_BYTES];
 
-spense_status noalloc_scratch(int dev, uint8_t** out) {
-  static std::mutex mu;
-  static std::vector<uint8_t*> addr;
-  std::lock_guard<std::mutex> lk(mu);
-  if (static_cast<int>(addr.size()) <= dev) addr.resize(dev + 1, nullptr);
-  if (addr[dev] == nullptr) {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-    addr[dev] = static_cast<uint8_t*>(p);
-  }
-  *out = addr[dev];
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch array for device `dev` (current), looked up
+// once per (device, context) with cudaGetSymbolAddress and cached. A context
+// handle that the driver reuses after a cudaDeviceReset would hit a stale
+// entry; the cache assumes each device keeps its context for the life of the
+// process (the runtime's primary context, as PyTorch uses it).
+spense_status noalloc_scratch(int dev, uint8_t** out) {
+  struct Slot {
+    int dev;
+    CUcontext ctx;
+    uint8_t* addr;
+  };
+  static std::mutex mu;
+  static std::vector<Slot> slots;
+  CUcontext ctx = nullptr;
+  if (CtxGetCurrentFn f = ctx_get_current()) f(&ctx);
+  std::lock_guard<std::mutex> lk(mu);
+  for (const Slot& sl : slots)
+    if (sl.dev == dev && sl.ctx == ctx) {
+      *out = sl.addr;
+      return SPENSE_OK;
+    }
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+  slots.push_back(Slot{dev, ctx, static_cast<uint8_t*>(p)});
+  *out = static_cast<uint8_t*>(p);
   return SPENSE_OK;
 }
 
@@ -654,12 +789,8 @@ spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int
   if (!aligned(W, 16) || (mask != nullptr && !aligned(mask, 16)) || !aligned(w_scale, 4))
     return fail(SPENSE_ERR_ALIGN, "W and mask must be 16-byte aligned, w_scale 4-byte aligned");
   if (dense_idx != nullptr) {
-    for (int64_t j = 0; j < Kd; ++j) {
-      if (dense_idx[j] < 0 || dense_idx[j] >= K)
-        return fail(SPENSE_ERR_DENSE_IDX, "dense_idx[%lld] = %d outside [0, K)", (long long)j, dense_idx[j]);
-      if (j > 0 && dense_idx[j] <= dense_idx[j - 1])
-        return fail(SPENSE_ERR_DENSE_IDX, "dense_idx is not strictly ascending at %lld", (long long)j);
-    }
+    const spense_status sd = check_dense_idx(dense_idx, Kd, K);
+    if (sd != SPENSE_OK) return sd;
   }
   int dev = 0;
   DeviceInfo info;
@@ -706,13 +837,8 @@ spense_status spense_pack(const uint8_t* W, const float* w_scale, int64_t N, int
     return cuda_fail(e, "pack allocation");
   }
   if (dense_idx != nullptr) {
-    std::vector<int32_t> perm;
-    perm.reserve(static_cast<size_t>(K));
-    std::vector<char> dense(static_cast<size_t>(K), 0);
-    for (int64_t j = 0; j < Kd; ++j) dense[static_cast<size_t>(dense_idx[j])] = 1;
-    for (int64_t k = 0; k < K; ++k)
-      if (!dense[static_cast<size_t>(k)]) perm.push_back(static_cast<int32_t>(k));
-    for (int64_t j = 0; j < Kd; ++j) perm.push_back(dense_idx[j]);
+    std::vector<int32_t> perm(static_cast<size_t>(K));
+    dense_block_order(dense_idx, Kd, K, perm.data());
     e = cudaMemcpyAsync(h->perm, perm.data(), perm.size() * 4, cudaMemcpyHostToDevice, stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(stream);  // `perm` is a host temporary
     h->perm_host = perm;
@@ -850,58 +976,13 @@ spense_status spense_gemm_grouped_ex(const spense_packed* const* Wps, int count,
   DeviceInfo info;
   spense_status st = check_gemm_args(Wps, count, M, workspace, &info);
   if (st != SPENSE_OK) return st;
+  for (int i = 0; i < count; ++i)
+    if (Wps[i] == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(SPENSE_ERR_UNSUPPORTED, "no CUDA device");
-  LaunchKey key;
-  key.device = dev;
-  key.count = count;
-  for (int i = 0; i < count; ++i) {
-    if (Wps[i] == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
-    key.ids[i] = Wps[i]->id;
-    key.Ys[i] = Ys[i];
-    key.ldy[i] = ldy != nullptr ? ldy[i] : Wps[i]->N;
-  }
-  key.M = M;
-  key.X = X;
-  key.x_scale = x_scale;
-  key.ws = workspace;
-  key.flags = flags;
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-  {
-    std::lock_guard<std::mutex> lk(g_launch_mu);
-    auto& cache = *g_launch_cache;
-    for (size_t i = 0; i < cache.size(); ++i) {
-      if (!(cache[i].key == key)) continue;
-      if (workspace_bytes < cache[i].ws_needed)
-        return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
-                    cache[i].ws_needed);
-      if (i != 0) std::rotate(cache.begin(), cache.begin() + static_cast<std::ptrdiff_t>(i),
-                              cache.begin() + static_cast<std::ptrdiff_t>(i) + 1);
-      st = enqueue_gemm(cache[0].launch, stream);
-      return st == SPENSE_OK ? ok() : st;
-    }
-  }
-  GemmPlan pl;
-  st = make_plan(Wps, count, M, info.sms, &pl);
-  if (st != SPENSE_OK) return st;
-  if (workspace_bytes < pl.ws.total_device)
-    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
-                pl.ws.total_device);
-  LaunchCacheEntry entry;
-  entry.key = key;
-  entry.ws_needed = pl.ws.total_device;
-  st = prepare_gemm(Wps, count, X, x_scale, M, Ys, static_cast<uint8_t*>(workspace), pl,
-                    (flags & SPENSE_GEMM_X_PACKED_ORDER) != 0u, ldy, &entry.launch);
-  if (st != SPENSE_OK) return st;
-  st = enqueue_gemm(entry.launch, stream);
-  if (st != SPENSE_OK) return st;
-  {
-    std::lock_guard<std::mutex> lk(g_launch_mu);
-    auto& cache = *g_launch_cache;
-    cache.insert(cache.begin(), entry);
-    if (cache.size() > kLaunchCacheSize) cache.pop_back();
-  }
-  return ok();
+  st = launch_grouped(Wps, count, X, x_scale, M, Ys, ldy, workspace, workspace_bytes, flags, dev, info,
+                      static_cast<cudaStream_t>(stream_v));
+  return st == SPENSE_OK ? ok() : st;
 }
 
 spense_status spense_quantize(const uint16_t* X, int64_t M, int64_t K, const spense_packed* order, uint8_t* Xq,
@@ -986,34 +1067,92 @@ spense_status spense_gemm(const spense_packed* Wp, const uint8_t* X, const float
   return spense_gemm_grouped(&Wp, 1, X, x_scale, M, &Y, workspace, workspace_bytes, stream_v);
 }
 
+spense_status spense_gemm_grouped_host(const spense_packed* const* Wps, int count, const uint8_t* X,
+                                       const float* x_scale, int64_t M, uint16_t* const* Ys, void* workspace,
+                                       size_t workspace_bytes, unsigned int flags, void* stream_v) {
+  const unsigned int known = SPENSE_GEMM_X_PACKED_ORDER | SPENSE_GEMM_HOST_X | SPENSE_GEMM_HOST_Y;
+  if ((flags & ~known) != 0u) return fail(SPENSE_ERR_ARG, "unknown flags %#x", flags);
+  if (X == nullptr || x_scale == nullptr || Ys == nullptr) return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
+  const bool host_x = (flags & SPENSE_GEMM_HOST_X) != 0u;
+  const bool host_y = (flags & SPENSE_GEMM_HOST_Y) != 0u;
+  if (!host_x && (!aligned(X, 16) || !aligned(x_scale, 4)))
+    return fail(SPENSE_ERR_ALIGN, "X must be 16-byte aligned, x_scale 4-byte aligned");
+  DeviceInfo info;
+  spense_status st = check_gemm_args(Wps, count, M, workspace, &info);
+  if (st != SPENSE_OK) return st;
+  for (int i = 0; i < count; ++i) {
+    if (Wps[i] == nullptr) return fail(SPENSE_ERR_ARG, "packed weight %d is NULL", i);
+    if (Ys[i] == nullptr) return fail(SPENSE_ERR_ARG, "Y[%d] is NULL", i);
+    if (!host_y && !aligned(Ys[i], 16)) return fail(SPENSE_ERR_ALIGN, "Y[%d] must be 16-byte aligned", i);
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(SPENSE_ERR_UNSUPPORTED, "no CUDA device");
+  GemmPlan pl;
+  st = make_plan(Wps, count, M, info.sms, &pl);
+  if (st != SPENSE_OK) return st;
+  const size_t need = (host_x || host_y) ? pl.ws.total_host : pl.ws.total_device;
+  if (workspace_bytes < need)
+    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes, need);
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const uint8_t* xd = X;
+  const float* sxd = x_scale;
+  if (host_x) {
+    uint8_t* xs = ws + pl.ws.stage_x_off;
+    float* sxs = reinterpret_cast<float*>(ws + pl.ws.stage_sx_off);
+    cudaError_t e = cudaMemcpyAsync(xs, X, static_cast<size_t>(M * Wps[0]->K), cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sxs, x_scale, static_cast<size_t>(M) * 4, cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    xd = xs;
+    sxd = sxs;
+  }
+  uint16_t* yd[kMaxGroup];
+  size_t y_off = pl.ws.stage_y_off;
+  for (int i = 0; i < count; ++i) {
+    if (host_y) {
+      yd[i] = reinterpret_cast<uint16_t*>(ws + y_off);
+      y_off += round_up(static_cast<size_t>(M * Wps[i]->N) * 2, 256);
+    } else {
+      yd[i] = Ys[i];
+    }
+  }
+  st = launch_grouped(Wps, count, xd, sxd, M, yd, nullptr, workspace, workspace_bytes,
+                      flags & SPENSE_GEMM_X_PACKED_ORDER, dev, info, stream);
+  if (st != SPENSE_OK) return st;
+  if (host_y) {
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < count && e == cudaSuccess; ++i)
+      e = cudaMemcpyAsync(Ys[i], yd[i], static_cast<size_t>(M * Wps[i]->N) * 2, cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  }
+  return ok();
+}
+
+size_t spense_gemm_grouped_host_workspace_size(const spense_packed* const* Wps, int count, int64_t M) {
+  int dev = 0;
+  DeviceInfo info;
+  if (current_device(&dev, &info) != SPENSE_OK) return 0;
+  GemmPlan pl;
+  if (make_plan(Wps, count, M, info.sms, &pl) != SPENSE_OK) return 0;
+  return pl.ws.total_host;
+}
+
 spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host, const float* x_scale_host,
                                int64_t M, uint16_t* Y_host, void* workspace, size_t workspace_bytes,
                                void* stream_v) {
-  if (X_host == nullptr || x_scale_host == nullptr || Y_host == nullptr)
-    return fail(SPENSE_ERR_ARG, "X, x_scale or Y is NULL");
-  DeviceInfo info;
-  spense_status st = check_gemm_args(&Wp, 1, M, workspace, &info);
+  if (Wp == nullptr) return fail(SPENSE_ERR_ARG, "Wp is NULL");
+  return spense_gemm_grouped_host(&Wp, 1, X_host, x_scale_host, M, &Y_host, workspace, workspace_bytes,
+                                  SPENSE_GEMM_HOST_X | SPENSE_GEMM_HOST_Y, stream_v);
+}
+
+spense_status spense_glu_order(int64_t I, const int32_t* dense_idx, int64_t Kd, int32_t* order) {
+  if (order == nullptr || (Kd > 0 && dense_idx == nullptr)) return fail(SPENSE_ERR_ARG, "order or dense_idx is NULL");
+  if (I < 1 || I > (1 << 20)) return fail(SPENSE_ERR_SHAPE, "I = %lld outside [1, 2^20]", (long long)I);
+  if (Kd < 0 || Kd > I) return fail(SPENSE_ERR_SHAPE, "Kd = %lld outside [0, I]", (long long)Kd);
+  const spense_status st = check_dense_idx(dense_idx, Kd, I);
   if (st != SPENSE_OK) return st;
-  GemmPlan pl;
-  st = make_plan(&Wp, 1, M, info.sms, &pl);
-  if (st != SPENSE_OK) return st;
-  if (workspace_bytes < pl.ws.total_host)
-    return fail(SPENSE_ERR_WORKSPACE, "workspace holds %zu bytes, %zu needed", workspace_bytes,
-                pl.ws.total_host);
-  cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* xd = ws + pl.ws.stage_x_off;
-  float* sxd = reinterpret_cast<float*>(ws + pl.ws.stage_sx_off);
-  uint16_t* yd = reinterpret_cast<uint16_t*>(ws + pl.ws.stage_y_off);
-  cudaError_t e = cudaMemcpyAsync(xd, X_host, static_cast<size_t>(M * Wp->K), cudaMemcpyHostToDevice, stream);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(sxd, x_scale_host, static_cast<size_t>(M) * 4, cudaMemcpyHostToDevice, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
-  st = run_gemm(&Wp, 1, xd, sxd, M, &yd, ws, pl, stream);
-  if (st != SPENSE_OK) return st;
-  e = cudaMemcpyAsync(Y_host, yd, static_cast<size_t>(M * Wp->N) * 2, cudaMemcpyDeviceToHost, stream);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
-  if (e != cudaSuccess) return cuda_fail(e, "device-to-host copy");
+  dense_block_order(dense_idx, Kd, I, order);
   return ok();
 }
 
@@ -1080,12 +1219,26 @@ spense_status spense_gemm_noalloc(const spense_packed* Wp, const uint8_t* X, con
   st = noalloc_scratch(dev, &ws);
   if (st != SPENSE_OK) return st;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
-  // The status word and the arrival counters must start at zero; the array
-  // keeps whatever the previous call left in it.
-  const cudaError_t e = cudaMemsetAsync(ws, 0, pl.ws.partials_off, stream);
+  // The arrival counters (and the rest of the header) must start at zero;
+  // the array keeps whatever the previous call left in it. The status word
+  // (the first 4 bytes) is left alone: a timeout stays recorded until
+  // spense_noalloc_status reads it.
+  const cudaError_t e = cudaMemsetAsync(ws + 4, 0, pl.ws.partials_off - 4, stream);
   if (e != cudaSuccess) return cuda_fail(e, "scratch clear");
   st = run_gemm(&Wp, 1, X, x_scale, M, &Y, ws, pl, stream);
   return st == SPENSE_OK ? ok() : st;
+}
+
+spense_status spense_noalloc_status(void* stream_v, uint32_t* status_out) {
+  if (status_out == nullptr) return fail(SPENSE_ERR_ARG, "status_out is NULL");
+  int dev = 0;
+  DeviceInfo info;
+  spense_status st = current_device(&dev, &info);
+  if (st != SPENSE_OK) return st;
+  uint8_t* ws = nullptr;
+  st = noalloc_scratch(dev, &ws);
+  if (st != SPENSE_OK) return st;
+  return spense_workspace_status(ws, stream_v, status_out);
 }
 
 }  // extern "C"

@@ -1,12 +1,15 @@
 """Run a few eager launches of one workload, for profilers.
 
     python -m dense_fp8_gemm_b200.run_case --workload attn32b --tokens 16 --repeat 3
+    python -m dense_fp8_gemm_b200.run_case --workload chain36b --tokens 16 --repeat 2
     python -m dense_fp8_gemm_b200.run_case --shape 51200x5120 --dense-frac 0.25 --tokens 16 --repeat 3
     python -m dense_fp8_gemm_b200.run_case --shape 5120x25600 --scattered --tokens 8192 --repeat 1
     python -m dense_fp8_gemm_b200.run_case --shape 25600x5120 --output-split --tokens 16 --repeat 1
 
 `attn32b` issues, per repeat, the two launches of one decoder layer's attention
-projections: q, k and v grouped on one input, then o_proj. `--shape NxK` runs a
+projections: q, k and v grouped on one input, then o_proj. `chain36b` issues
+the four launches of one layer of the 36B-class stack (q/k/v grouped, o_proj,
+gate+up, down), its weights drawn on the GPU as the benchmark draws them. `--shape NxK` runs a
 single GEMM: with `--scattered` its dense columns are a seeded random set
 (SpenseGPT+, so each call gathers X into the packed column order first); with
 `--output-split` its 2:4 rows and its dense rows (a seeded random set) are
@@ -26,7 +29,7 @@ from . import spense, synth, workloads
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--workload", default=None, choices=[None, "attn32b"])
+    ap.add_argument("--workload", default=None, choices=[None, "attn32b", "chain36b"])
     ap.add_argument("--shape", default=None, help="NxK for a single GEMM")
     ap.add_argument("--dense-frac", type=float, default=0.25)
     ap.add_argument("--tokens", type=int, default=16)
@@ -60,6 +63,18 @@ def main(argv=None):
             grp = [spense.pack(Wd, sd, Kd=Kd)]
         X, s_x = synth.quantize_rows(synth.normal(1, 3, (M, K), 1.0))
         launches.append((grp, torch.from_numpy(X).to(dev), torch.from_numpy(s_x).to(dev)))
+    elif args.workload == "chain36b":
+        wl = workloads.CHAIN36B
+
+        def packed_dev(i):
+            _, N, K = wl.shapes[i]
+            q, sc = synth.device_fp8_rows(wl.seed, workloads.weight_id(i, 0), (N, K), wl.w_std, dev)
+            return spense.pack(q, sc, Kd=workloads.dense_count(K, args.dense_frac))
+
+        for grp_idx in ((0, 1, 2), (3,), (4,), (5,)):
+            X, s_x = workloads.make_activations(wl, grp_idx[0], M)
+            launches.append(([packed_dev(i) for i in grp_idx], torch.from_numpy(X).to(dev),
+                             torch.from_numpy(s_x).to(dev)))
     else:
         wl = workloads.ATTN32B
         qkv = [packed(wl, i) for i in range(3)]

@@ -13,7 +13,7 @@ import os
 import numpy as np
 import torch
 
-from .build import LIB_PATH
+from .build import LIB_PATH, TEST_LIB_PATH
 
 SPENSE_OK = 0
 STATUS_NAMES = {
@@ -30,11 +30,14 @@ SYMBOLS = (
     "spense_workspace_status", "spense_last_error", "spense_version", "spense_gemm_noalloc",
     "spense_gemm_grouped", "spense_gemm_grouped_workspace_size", "spense_gemm_grouped_ex",
     "spense_quantize", "spense_score_glu", "spense_score_workspace_size", "spense_select_dense",
-    "spense_pack_rows", "spense_plan_shapes",
+    "spense_pack_rows", "spense_plan_shapes", "spense_gemm_grouped_host",
+    "spense_gemm_grouped_host_workspace_size", "spense_glu_order", "spense_noalloc_status",
 )
 GEMM_X_PACKED_ORDER = 1
+GEMM_HOST_X = 2
+GEMM_HOST_Y = 4
 MAX_GROUP = 4
-NOALLOC_SCRATCH_BYTES = 8 << 20
+NOALLOC_SCRATCH_BYTES = (8 << 20) + (64 << 10)
 
 
 class SpenseError(RuntimeError):
@@ -67,14 +70,20 @@ class PlanInfo(ctypes.Structure):
                 ("workspace_bytes", ctypes.c_uint64), ("cta_start", ctypes.c_int32 * (PLAN_MAX_GRID + 1))]
 
 
+def lib_path() -> str:
+    """libspense.so, or its test-hook build when SPENSE_TEST_HOOKS=1 (failure tests only)."""
+    return TEST_LIB_PATH if os.environ.get("SPENSE_TEST_HOOKS") == "1" else LIB_PATH
+
+
 def lib() -> ctypes.CDLL:
     """Load libspense.so (built in-tree by dense_fp8_gemm_b200.build)."""
     global _lib
     if _lib is not None:
         return _lib
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"libspense.so not found at {LIB_PATH}; run dense_fp8_gemm_b200.build.build()")
-    L = ctypes.CDLL(LIB_PATH)
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{os.path.basename(path)} not found at {path}; run dense_fp8_gemm_b200.build.build()")
+    L = ctypes.CDLL(path)
     P, I64, SZ, U32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_uint32
     L.spense_pack.argtypes = [P, P, I64, I64, P, P, I64, U32, P, ctypes.POINTER(P)]
     L.spense_gemm.argtypes = [P, P, P, I64, P, P, SZ, P]
@@ -99,10 +108,17 @@ def lib() -> ctypes.CDLL:
     L.spense_score_workspace_size.argtypes = [I64, I64]
     L.spense_score_workspace_size.restype = SZ
     L.spense_select_dense.argtypes = [P, I64, I64, P, P]
+    L.spense_gemm_grouped_host.argtypes = [ctypes.POINTER(P), ctypes.c_int, P, P, I64, ctypes.POINTER(P), P, SZ,
+                                           U32, P]
+    L.spense_gemm_grouped_host_workspace_size.argtypes = [ctypes.POINTER(P), ctypes.c_int, I64]
+    L.spense_gemm_grouped_host_workspace_size.restype = SZ
+    L.spense_glu_order.argtypes = [I64, P, I64, P]
+    L.spense_noalloc_status.argtypes = [P, ctypes.POINTER(U32)]
     L.spense_last_error.restype = ctypes.c_char_p
     L.spense_version.restype = ctypes.c_char_p
     for name in ("spense_pack", "spense_gemm", "spense_gemm_host", "spense_free", "spense_get_info",
-                 "spense_workspace_status", "spense_gemm_noalloc", "spense_gemm_grouped"):
+                 "spense_workspace_status", "spense_gemm_noalloc", "spense_gemm_grouped",
+                 "spense_gemm_grouped_host", "spense_glu_order", "spense_noalloc_status"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -356,6 +372,63 @@ class PreparedGrouped:
             _check(code, "spense_gemm_grouped_ex")
 
 
+def grouped_host_workspace_size(pws, M: int) -> int:
+    n = lib().spense_gemm_grouped_host_workspace_size(_handles(pws), len(pws), M)
+    if n == 0:
+        _check(1, "spense_gemm_grouped_host_workspace_size")
+    return int(n)
+
+
+def _ptr(t: torch.Tensor, dtype, name: str, host: bool):
+    if host:
+        if t.is_cuda or t.dtype != dtype or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {dtype} host tensor")
+        return ctypes.c_void_p(t.data_ptr())
+    return _dev_ptr(t, dtype, name)
+
+
+class PreparedGroupedHost:
+    """spense_gemm_grouped_host with its arguments marshalled once: X (and
+    x_scale) in host memory when flags has GEMM_HOST_X, the outputs in host
+    memory when it has GEMM_HOST_Y (the call then synchronizes the stream).
+    The tensors must stay alive and in place."""
+
+    def __init__(self, pws, X: torch.Tensor, x_scale: torch.Tensor, Ys, workspace: torch.Tensor, flags: int):
+        hx, hy = bool(flags & GEMM_HOST_X), bool(flags & GEMM_HOST_Y)
+        self._keep = (list(pws), X, x_scale, list(Ys), workspace)
+        yarr = (ctypes.c_void_p * len(pws))()
+        for i, Y in enumerate(Ys):
+            yarr[i] = _ptr(Y, torch.bfloat16, f"Y[{i}]", hy).value
+        self._fn = lib().spense_gemm_grouped_host
+        self._args = (_handles(pws), len(pws), _ptr(X, torch.uint8, "X", hx),
+                      _ptr(x_scale, torch.float32, "x_scale", hx), X.shape[0], yarr,
+                      _dev_ptr(workspace, torch.uint8, "workspace"), workspace.numel(), int(flags))
+
+    def __call__(self, stream=None):
+        code = self._fn(*self._args, _stream(stream))
+        if code != SPENSE_OK:
+            _check(code, "spense_gemm_grouped_host")
+
+
+def gemm_grouped_host(pws, X: torch.Tensor, x_scale: torch.Tensor, Ys, workspace: torch.Tensor, flags: int,
+                      stream=None):
+    """spense_gemm_grouped_host: one grouped launch whose input (GEMM_HOST_X),
+    outputs (GEMM_HOST_Y) or both live in host memory; the copies run inside
+    the call. Returns Ys."""
+    PreparedGroupedHost(pws, X, x_scale, Ys, workspace, flags)(stream)
+    return Ys
+
+
+def glu_order(I: int, dense_idx) -> np.ndarray:
+    """spense_glu_order: the other intermediate indices ascending, then the
+    dense set (the packed column order of a weight packed with that set)."""
+    idx = np.ascontiguousarray(np.asarray(dense_idx, dtype=np.int32))
+    out = np.empty((I,), dtype=np.int32)
+    _check(lib().spense_glu_order(int(I), idx.ctypes.data_as(ctypes.c_void_p) if idx.size else None, idx.size,
+                                  out.ctypes.data_as(ctypes.c_void_p)), "spense_glu_order")
+    return out
+
+
 def quantize(X: torch.Tensor, order: PackedWeight | None = None, Xq: torch.Tensor | None = None,
              x_scale: torch.Tensor | None = None, stream=None):
     """spense_quantize: per-token FP8 quantisation of bf16 activations X [M, K]
@@ -385,6 +458,14 @@ def gemm_noalloc(pw: PackedWeight, X: torch.Tensor, x_scale: torch.Tensor, Y: to
                                      _dev_ptr(Y, torch.bfloat16, "Y"), _stream(stream))
     _check(code, "spense_gemm_noalloc")
     return Y
+
+
+def noalloc_status(stream=None) -> int:
+    """Reads and clears the status word of the noalloc scratch on the current
+    device (0 = every noalloc GEMM since the last read completed normally)."""
+    out = ctypes.c_uint32()
+    _check(lib().spense_noalloc_status(_stream(stream), ctypes.byref(out)), "spense_noalloc_status")
+    return int(out.value)
 
 
 def workspace_status(workspace: torch.Tensor, stream=None) -> int:

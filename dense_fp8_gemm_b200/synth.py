@@ -40,6 +40,32 @@ def quantize_rows(x: np.ndarray):
     return q, s
 
 
+def device_fp8_rows(seed: int, tensor_id: int, shape, std: float, device, outliers: bool = False):
+    """The recipe of ``normal`` (+ ``weight_outliers`` when `outliers`) +
+    ``quantize_rows`` drawn on the GPU, for weights too large to draw on the
+    host in reasonable time (a 64-layer decoder stack): N(0, std) from torch's
+    counter-based Philox generator on `device`, seeded from (seed, tensor_id);
+    with `outliers`, a Bernoulli(0.01) subset of the entries (a second draw of
+    the same generator) multiplied by 20; then per-row absmax FP8 e4m3
+    quantisation (s = absmax / 448, 1 for an all-zero row; round to nearest
+    even, saturated to +-448). Same distribution as the host recipe, not the
+    same values. Returns (q uint8 [rows, cols], s float32 [rows]) on `device`."""
+    g = torch.Generator(device=device)
+    g.manual_seed((int(seed) << 32) ^ int(tensor_id))
+    w = torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32)
+    w.mul_(std)
+    if outliers:
+        hit = torch.rand(tuple(shape), generator=g, device=device, dtype=torch.float32) < 0.01
+        w[hit] *= 20.0
+        del hit
+    amax = w.abs().amax(dim=1)
+    s = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
+    w.div_(s[:, None]).clamp_(-E4M3_MAX, E4M3_MAX)
+    q = w.to(torch.float8_e4m3fn).view(torch.uint8)
+    del w
+    return q, s.to(torch.float32)
+
+
 def weight_outliers(seed: int, tensor_id: int, w: np.ndarray, frac: float = 0.01,
                     factor: float = 20.0) -> np.ndarray:
     """Multiply a Bernoulli(frac) subset of the entries by `factor`."""

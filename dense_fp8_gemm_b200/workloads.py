@@ -7,7 +7,9 @@ every tensor is drawn by ``synth`` from the seeds below.
 
 Tensor ids: weight of shape i -> 100 + 10 i; its outlier stream -> 101 + 10 i;
 its dense-index score -> 102 + 10 i; activations for (shape i, batch M) ->
-10000 + 1000 i + M, their outlier stream -> 10000 + 1000 i + M + 500.
+10000 + 1000 i + M, their outlier stream -> 10000 + 1000 i + M + 500. Layer L
+of a multi-layer workload adds 1000000 L to its weight ids (layer 0 is the
+single-layer weight).
 """
 from __future__ import annotations
 
@@ -72,13 +74,22 @@ class Weight:
         return self.W.shape[1]
 
 
-def make_weight(wl: Workload, i: int, dense_frac: float | None = None) -> Weight:
+def weight_id(i: int, layer: int = 0) -> int:
+    """Tensor id of the weight of shape i in layer `layer`."""
+    return 100 + 10 * i + 1000000 * layer
+
+
+def make_weight(wl: Workload, i: int, dense_frac: float | None = None, layer: int = 0, rows=None) -> Weight:
+    """The weight of shape i (layer `layer`), quantised per row. `rows`: draw a
+    matrix of only that many rows (a sample with the shape's columns and
+    distribution, from its own stream)."""
     label, N, K = wl.shapes[i]
     df = wl.dense_fracs[0] if dense_frac is None else dense_frac
     Kd = dense_count(K, df)
-    w = synth.normal(wl.seed, 100 + 10 * i, (N, K), wl.w_std)
+    tid = weight_id(i, layer) + (500000 if rows is not None else 0)
+    w = synth.normal(wl.seed, tid, (N if rows is None else rows, K), wl.w_std)
     if wl.outliers:
-        w = synth.weight_outliers(wl.seed, 101 + 10 * i, w)
+        w = synth.weight_outliers(wl.seed, tid + 1, w)
     q, s = synth.quantize_rows(w)
     del w
     idx = synth.scored_dense_idx(wl.seed, 102 + 10 * i, K, Kd) if wl.scattered else None

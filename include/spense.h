@@ -176,13 +176,17 @@ SPENSE_API spense_status spense_gemm_grouped(const spense_packed* const* Wps, in
 
 SPENSE_API size_t spense_gemm_grouped_workspace_size(const spense_packed* const* Wps, int count, int64_t M);
 
-/* Flags of spense_gemm_grouped_ex. */
+/* Flags of spense_gemm_grouped_ex and spense_gemm_grouped_host. */
 enum {
   /* X (and x_scale) are already in the packed column order of the weights
    * (sparse columns ascending, then the dense columns in dense_idx order), as
    * spense_quantize writes them when given one of the weights as `order`; the
    * GEMM then skips its own gather. No effect for a tail dense set. */
-  SPENSE_GEMM_X_PACKED_ORDER = 1u
+  SPENSE_GEMM_X_PACKED_ORDER = 1u,
+  /* spense_gemm_grouped_host only: X and x_scale are in HOST memory. */
+  SPENSE_GEMM_HOST_X = 2u,
+  /* spense_gemm_grouped_host only: the outputs Ys are in HOST memory. */
+  SPENSE_GEMM_HOST_Y = 4u
 };
 
 /*
@@ -277,17 +281,67 @@ SPENSE_API spense_status spense_select_dense(const float* score, int64_t I, int6
                                              void* stream);
 
 /*
+ * spense_gemm_grouped_host — spense_gemm_grouped with its input, its outputs or
+ * both in HOST memory; the copies between host and device run inside the call,
+ * on `stream`, through staging areas of the workspace. The GEMM itself is the
+ * one of Technical Summary §2.A / §2.B described above.
+ *   flags  SPENSE_GEMM_HOST_X: X [M][K] and x_scale [M] are host pointers,
+ *          copied to the device before the GEMM (a pageable buffer may be
+ *          reused when the call returns; a pinned one must stay unchanged
+ *          until the stream has passed the call).
+ *          SPENSE_GEMM_HOST_Y: Ys[i] [M][N_i] are host pointers; the outputs
+ *          are copied back and the call synchronizes `stream` before
+ *          returning. Without it the call is asynchronous, like
+ *          spense_gemm_grouped.
+ *          SPENSE_GEMM_X_PACKED_ORDER as for spense_gemm_grouped_ex.
+ *          With neither HOST flag it is spense_gemm_grouped_ex without ldy.
+ *   workspace  at least spense_gemm_grouped_host_workspace_size(Wps, count, M)
+ *          bytes when a HOST flag is set (else the grouped size), same rules
+ *          as spense_gemm. Device-side inputs and outputs keep the alignment
+ *          rules of spense_gemm; host ones have none.
+ * A typical use is a stack of layers issued in stream order: the first call
+ * takes the host input (HOST_X), the middle ones run on device buffers, and
+ * the last returns the host output (HOST_Y).
+ * Errors: as spense_gemm_grouped, plus ARG for unknown flags.
+ */
+SPENSE_API spense_status spense_gemm_grouped_host(const spense_packed* const* Wps, int count, const uint8_t* X,
+                                                  const float* x_scale, int64_t M, uint16_t* const* Ys,
+                                                  void* workspace, size_t workspace_bytes, unsigned int flags,
+                                                  void* stream);
+
+SPENSE_API size_t spense_gemm_grouped_host_workspace_size(const spense_packed* const* Wps, int count, int64_t M);
+
+/*
  * spense_gemm_host — the same GEMM on HOST buffers: copies X [M][K] and
  * x_scale [M] from host memory into the workspace, runs spense_gemm, copies Y
  * [M][N] back to host memory and synchronizes `stream` before returning.
  * Host buffers should be pinned for asynchronous copies. workspace must hold
  * spense_gemm_host_workspace_size(Wp, M) bytes (zero-filled before first use).
+ * It is spense_gemm_grouped_host over one weight with both HOST flags.
  */
 SPENSE_API spense_status spense_gemm_host(const spense_packed* Wp, const uint8_t* X_host,
                                const float* x_scale_host, int64_t M, uint16_t* Y_host,
                                void* workspace, size_t workspace_bytes, void* stream);
 
 SPENSE_API size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64_t M);
+
+/*
+ * spense_glu_order — the order in which SpenseGPT+ lays out the intermediate
+ * indices of a GLU MLP once its dense set is chosen (Technical Summary §2.B:
+ * the selected dense indices are permuted into one contiguous block; the
+ * permutation leaves the MLP's output unchanged): every index in [0, I) that is
+ * not in dense_idx, ascending, then dense_idx. It is also the packed column
+ * order spense_pack gives a weight packed with this dense set. Pack the gate
+ * and up rows with spense_pack_rows(rows = order) to make their outputs arrive
+ * in this order, so down (packed with the same dense set) reads them with
+ * SPENSE_GEMM_X_PACKED_ORDER and no gather.
+ *   I          1 .. 2^20 intermediate indices.
+ *   dense_idx  HOST int32 [Kd], strictly ascending in [0, I) (NULL if Kd == 0).
+ *   Kd         0 .. I.
+ *   order      HOST int32 [I] (caller-owned), written on success.
+ * Host only: needs no device. Errors: ARG, SHAPE, DENSE_IDX.
+ */
+SPENSE_API spense_status spense_glu_order(int64_t I, const int32_t* dense_idx, int64_t Kd, int32_t* order);
 
 /*
  * spense_gemm_noalloc — the same GEMM as spense_gemm, for callers that must not
@@ -299,24 +353,35 @@ SPENSE_API size_t spense_gemm_host_workspace_size(const spense_packed* Wp, int64
  * counterpart to this entry point; it is a deployment convenience.
  *
  * Instead of a caller workspace it uses one fixed scratch array of
- * SPENSE_NOALLOC_SCRATCH_BYTES that the library places in device memory; every
- * GPU that loads the library holds it until the process exits. Calls whose
- * workspace need (spense_gemm_workspace_size) exceeds it are rejected with
- * SPENSE_ERR_WORKSPACE; decode-sized calls (up to a few dozen tokens on the
- * 32B/36B-class shapes) fit. The call allocates nothing: no cudaMalloc, no
+ * SPENSE_NOALLOC_SCRATCH_BYTES (8 MiB + 64 KiB) that the library places in
+ * device memory; every GPU that loads the library holds it until the process
+ * exits. Calls whose workspace need (spense_gemm_workspace_size) exceeds it
+ * are rejected with SPENSE_ERR_WORKSPACE. On a B200 (148 SMs) every weight
+ * of the 32B- and 36B-class decoder shapes (K <= 27648, tail dense set) fits
+ * for M <= 32 tokens; a SpenseGPT+ weight also stages M x K gathered
+ * activation bytes there. The call allocates nothing: no cudaMalloc, no
  * cudaFree, no allocating library routine.
  *
  * The first call on a device looks up the array's device address (with that
- * device current), so make that first call before any stream capture. Every
- * call clears the array's status word and counters on `stream` before the
- * GEMM. All calls share the one array: calls whose execution can overlap on the
- * GPU (different streams without ordering between them) race on it and give
- * wrong results; serialize them. Arguments, layouts and the remaining errors
- * are those of spense_gemm. Asynchronous on `stream`.
+ * device current), so make that first call before any stream capture; the
+ * address is cached per device and context. Every call clears the array's
+ * arrival counters on `stream` before the GEMM. A wait that gave up on the
+ * device is recorded in the array's status word, which stays set until
+ * spense_noalloc_status reads and clears it. All calls share the one array:
+ * calls whose execution can overlap on the GPU (different streams without
+ * ordering between them) race on it and give wrong results; serialize them.
+ * Arguments, layouts and the remaining errors are those of spense_gemm.
+ * Asynchronous on `stream`.
  */
-#define SPENSE_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define SPENSE_NOALLOC_SCRATCH_BYTES ((8u << 20) + (64u << 10))
 SPENSE_API spense_status spense_gemm_noalloc(const spense_packed* Wp, const uint8_t* X, const float* x_scale,
                                              int64_t M, uint16_t* Y, void* stream);
+
+/* Reads and clears the status word of spense_gemm_noalloc's scratch array on
+ * the current device, as spense_workspace_status does for a workspace: 0 when
+ * every noalloc GEMM since the last read completed normally, else an OR of
+ * SPENSE_DEVICE_* codes. Synchronizes `stream`. Errors: ARG, UNSUPPORTED, CUDA. */
+SPENSE_API spense_status spense_noalloc_status(void* stream, uint32_t* status_out);
 
 /* Releases the handle and its device buffers (stream-ordered on the stream the
  * handle was packed on). NULL is accepted. */

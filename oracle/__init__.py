@@ -60,6 +60,8 @@ def _load():
     lib.oracle_score_glu.restype = ctypes.c_int
     lib.oracle_select_top.argtypes = [P, I64, I64, P]
     lib.oracle_select_top.restype = ctypes.c_int
+    lib.oracle_hardware_concurrency.argtypes = []
+    lib.oracle_hardware_concurrency.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -245,6 +247,11 @@ def glu_order(I, dense_idx):
     d = np.asarray(dense_idx, dtype=np.int64)
     rest = np.setdiff1d(np.arange(I, dtype=np.int64), d)
     return np.concatenate([rest, np.sort(d)])
+
+
+def hardware_concurrency() -> int:
+    """std::thread::hardware_concurrency() of the host the oracle runs on."""
+    return int(_load().oracle_hardware_concurrency())
 
 
 def within_tolerance(y, yref, bound, rel=4e-3, absb=1e-5):

@@ -152,6 +152,10 @@ float bf16_to_float(uint16_t b) {
 
 extern "C" {
 
+// Threads the host offers (std::thread::hardware_concurrency), reported beside
+// the oracle's timings; 0 when unknown.
+int oracle_hardware_concurrency(void) { return static_cast<int>(std::thread::hardware_concurrency()); }
+
 // Decode all 256 e4m3 bytes (R1).
 void oracle_e4m3_table(double* out256) {
   for (int b = 0; b < 256; ++b) out256[b] = decode_e4m3(static_cast<uint8_t>(b));

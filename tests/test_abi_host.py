@@ -185,3 +185,23 @@ def test_pack_rows_rejects_bad_arguments(L):
     assert call(W=0x1004) == 3
     assert call() == 1  # rows[1] = 5 is outside [0, 4)
     assert b"rows[1]" in L.spense_last_error()
+
+
+def test_glu_order_matches_the_oracle_reading():
+    """spense_glu_order (host only) against the oracle's independent restatement
+    of the SpenseGPT+ layout: the other indices ascending, then the dense set."""
+    import oracle
+    rng = np.random.default_rng(11)
+    for I, kd in ((1, 0), (1, 1), (10, 3), (4096, 1024), (25600, 6400), (27648, 0), (64, 64)):
+        d = np.sort(rng.choice(I, kd, replace=False)).astype(np.int32)
+        got = spense.glu_order(I, d)
+        assert got.dtype == np.int32
+        assert np.array_equal(got, oracle.glu_order(I, d))
+
+
+def test_glu_order_rejects_bad_sets(L):
+    for I, d, code in ((8, [3, 3], 5), (8, [5, 2], 5), (8, [8], 5), (8, [-1], 5), (0, [], 2),
+                       (4, [0, 1, 2, 3, 3], 2)):
+        with pytest.raises(spense.SpenseError) as e:
+            spense.glu_order(I, d)
+        assert e.value.code == code, (I, d, e.value)

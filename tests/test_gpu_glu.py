@@ -7,7 +7,8 @@ SpenseGPT+ permutation folded upstream (Technical Summary §2A, §2B).
 - GLU policy: gate and up output-split (four members, one launch), down
   input-split with a scattered dense set. Folding the permutation: gate and
   up rows are packed in the GLU order (sparse indices, then dense ones), so
-  their outputs arrive permuted and down runs without its gather.
+  their outputs arrive permuted and down runs without its gather. The order
+  comes from the library (spense_glu_order); the oracle only checks results.
 """
 import numpy as np
 import pytest
@@ -36,7 +37,7 @@ def test_output_split_matches_oracle(N, K, M, frac):
     W, s_w = synth.quantize_rows(synth.normal(N, 1, (N, K), 0.02))
     X, s_x = synth.quantize_rows(synth.normal(N, 2, (M, K), 1.0))
     dense_rows = dense_rows_for(N, frac, N)
-    order = oracle.glu_order(N, dense_rows)           # sparse rows, then dense rows
+    order = spense.glu_order(N, dense_rows)           # sparse rows, then dense rows (the library's order)
     Ns = N - dense_rows.size
     Wd, sd = torch.from_numpy(W).cuda(), torch.from_numpy(s_w).cuda()
     sp = spense.pack(Wd, sd, Kd=0, rows=order[:Ns])
@@ -75,7 +76,7 @@ def test_glu_policy_with_the_permutation_folded_upstream(I, H, M):
     x, s_x = synth.quantize_rows(synth.normal(7, 4, (M, H), 1.0))
     Nd = I // 4
     D = np.sort(g.choice(I, Nd, replace=False)).astype(np.int32)   # the SpenseGPT+ dense set
-    pi = oracle.glu_order(I, D)
+    pi = spense.glu_order(I, D)                      # the library's GLU order
     Ns = I - Nd
     dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
     # gate and up: output-split, rows in the GLU order (dense rows last); one launch of four members

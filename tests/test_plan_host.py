@@ -7,7 +7,7 @@ cluster choices that the measurements justify are the ones made.
 """
 import pytest
 
-from dense_fp8_gemm_b200 import spense
+from dense_fp8_gemm_b200 import spense, workloads
 
 SMS = 148
 SMEM_MAX = 232448
@@ -83,8 +83,9 @@ def test_plan_invariants(name, M):
     # tensor memory: a power of two from 32 columns holding the accumulators and the metadata
     assert p["tmem_cols"] in (32, 64, 128, 256, 512)
     assert p["nacc"] * npad + 16 <= p["tmem_cols"] <= 512 // cps
-    # the workspace holds every CTA's two fp32 partial slots
-    assert p["workspace_bytes"] >= grid * 2 * npad * 128 * 4
+    # stream-K: the workspace holds every CTA's two fp32 partial slots (a cluster reduces in shared memory)
+    if S == 1:
+        assert p["workspace_bytes"] >= grid * 2 * npad * 128 * 4
     assert p["l2_prefetch"] == (4 if S > 1 else 0)
 
 
@@ -104,13 +105,29 @@ def test_plan_choices(name, M, npad, S, cps):
 
 
 def test_plan_workspace_layout():
-    # status header (256 B), one arrival counter per tile (256-byte rounded), two fp32 partial slots of
-    # 128 rows x npad tokens per CTA; no gather buffer for a tail dense region
+    # status header (256 B), one arrival counter per tile (256-byte rounded), and for stream-K two fp32
+    # partial slots of 128 rows x npad tokens per CTA (none for a cluster split, which reduces in shared
+    # memory); no gather buffer for a tail dense region
+    seen = set()
     for name in ("qkv", "gateup", "down", "split"):
         for M in (1, 16, 256, 600):
             p = spense.plan_shapes(SHAPES[name], M, SMS)
             counters = -(-p["tiles"] * 4 // 256) * 256
-            assert p["workspace_bytes"] == 256 + counters + p["grid"] * 2 * p["npad"] * 128 * 4
+            partials = 0 if p["cluster"] > 1 else p["grid"] * 2 * p["npad"] * 128 * 4
+            assert p["workspace_bytes"] == 256 + counters + partials
+            seen.add(p["cluster"] > 1)
+    assert seen == {True, False}
+
+
+def test_noalloc_scratch_fits_the_decoder_shapes_up_to_32_tokens():
+    """spense_gemm_noalloc's fixed scratch holds the workspace of every 32B- and
+    36B-class decoder weight (tail dense set) for M <= 32 on a 148-SM B200, as
+    its header states."""
+    for wl in (workloads.ATTN32B, workloads.FFN32B, workloads.CHAIN36B):
+        for _, N, K in wl.shapes:
+            for M in range(1, 33):
+                p = spense.plan_shapes([(N, K, workloads.dense_count(K, 0.25))], M, SMS)
+                assert p["workspace_bytes"] <= spense.NOALLOC_SCRATCH_BYTES, (wl.name, N, K, M)
 
 
 def test_plan_rejects_bad_shapes():

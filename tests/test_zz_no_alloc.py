@@ -5,9 +5,11 @@ that owns every allocation and gives plugins none, or a serving loop that bans
 cudaMalloc after start-up), so they cannot pass a workspace. spense_gemm_noalloc
 uses the library's own fixed scratch array instead. This test calls it through
 the C ABI twice in a row (the second call finds the first call's leftovers in
-the shared array) and checks both outputs against the workspace entry point
-within the tolerance the parity tests use. It runs last so that a failure here
-never hides the result of another test, and it works alone in a fresh process.
+the shared array) and checks both outputs bit for bit against the workspace
+entry point (the same plan and kernel) and against the oracle within the
+parity tolerance, and that the calls leave the device's free memory
+unchanged. It runs last so that a failure here never hides the result of
+another test, and it works alone in a fresh process.
 """
 import numpy as np
 import pytest
@@ -18,12 +20,11 @@ from dense_fp8_gemm_b200 import spense, synth
 
 pytestmark = pytest.mark.gpu
 
-REL, ABS = 4e-3, 1e-5
-
 CASES = [
     # M, N, K, Kd, scattered
     (8, 256, 512, 128, False),
     (16, 8192, 5120, 1280, False),     # q_proj at decode: tiles shared by several CTAs
+    (24, 8192, 5120, 1280, False),     # q_proj, 24 tokens: the largest plan of the 32B shapes
     (1, 1024, 5120, 1280, False),
     (24, 2048, 4096, 1024, True),      # SpenseGPT+ gather into the scratch
 ]
@@ -42,15 +43,23 @@ def test_noalloc_matches_workspace_entry_point(M, N, K, Kd, scattered):
     Xd, sxd = _dev(X), _dev(s_x)
     Y_ws = spense.gemm(pw, Xd, sxd)  # the existing entry point, with its own workspace
     keep = oracle.pack(W, dense_idx=idx, Kd=Kd)["keep"]
-    _, bound = oracle.gemm(X, s_x, W, s_w, keep=keep)  # sum_k |w_k x_k| scaled, per output
-    y_ws = Y_ws.float().cpu().numpy().astype(np.float64)
+    yref, bound = oracle.gemm(X, s_x, W, s_w, keep=keep)
+    assert oracle.within_tolerance(Y_ws.float().cpu().numpy(), yref, bound).all()
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    spense.gemm_noalloc(pw, Xd, sxd, Y)  # first call on this device: looks up the scratch address
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
     for call in range(2):
-        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        Y.fill_(float("nan"))
         spense.gemm_noalloc(pw, Xd, sxd, Y)
         torch.cuda.synchronize()
+        # the same plan and kernel as the workspace entry point: bit for bit the same output
+        assert torch.equal(Y.view(torch.int16), Y_ws.view(torch.int16)), f"call {call}: differs from spense_gemm"
         y = Y.float().cpu().numpy().astype(np.float64)
-        ok = np.abs(y - y_ws) <= REL * np.abs(y_ws) + ABS * bound
+        ok = oracle.within_tolerance(y, yref, bound)
         assert ok.all(), f"call {call}: {int((~ok).sum())} of {ok.size} outputs outside tolerance"
+    assert torch.cuda.mem_get_info()[0] == free_before, "device memory was allocated by the noalloc calls"
+    assert spense.noalloc_status() == 0
     pw.free()
 
 
