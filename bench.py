@@ -433,7 +433,11 @@ def run_spense(args):
     ws_bytes = max(spense.grouped_host_workspace_size([arms[a][0][i] for i in g], m)
                    for a in arms for g in groups for m in Ms)
     ws = spense.new_workspace(ws_bytes, dev)
-    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    # Everything runs on one side stream (graphs cannot be captured on the
+    # legacy default stream); events and graph replays use it as the current stream.
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.set_stream(stream)
 
     def prepared(arm, M, gis=None):
         """PreparedGrouped calls of one step (layer by layer) at M tokens."""
