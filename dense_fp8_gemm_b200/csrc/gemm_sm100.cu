@@ -63,6 +63,7 @@ struct alignas(8) Barriers {
   uint64_t acc_empty[2];
   uint64_t peer_done;  // cluster mode, rank 0: completes when every peer's partial has landed
   uint64_t ack;        // cluster mode, peers: rank 0 has received this CTA's partial
+  uint64_t peer_full[kMaxStages];  // pair mode, even CTA: the odd CTA's stage has landed
   uint32_t tmem_base;
   int abort_flag;
   int fix_flag;
@@ -201,6 +202,14 @@ struct BlockWalker {
     member = member_of(p, n_tile);
     local_tile = n_tile - p.mem[member].tile_begin;
   }
+  // Row tile of the member whose weights this CTA streams: the tile itself,
+  // or in pair mode tile 2 x (pair tile) + the CTA's rank in the pair (the
+  // odd CTA of a member's last pair past its row count re-reads the last
+  // tile; its results are not stored).
+  __device__ int weight_tile(const GemmParams& p, uint32_t prank) const {
+    if (!p.pair) return local_tile;
+    return min(2 * local_tile + static_cast<int>(prank), p.mem[member].row_tiles - 1);
+  }
   __device__ void advance(const GemmParams& p) {
     if (++j == j1) {
       ++u;
@@ -225,6 +234,10 @@ __device__ __forceinline__ uint16_t to_bf16_bits(float v) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
 
+// kPair: the pair-mode instantiation. A kernel holding tcgen05 cta_group::2
+// instructions can only be launched as clusters of CTA pairs, so the
+// single-CTA modes (stream-K, cluster K-split) use the other instantiation.
+template <bool kPair>
 __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     spense_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -236,13 +249,21 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = blockIdx.x;
+  // Pair mode: CTAs 2u and 2u + 1 (one cluster) are work unit u; the even
+  // CTA (rank 0) issues the pair's MMAs. Otherwise every CTA is a work unit.
+  constexpr bool pair = kPair;
+  const uint32_t prank = pair ? ptx::cluster_ctarank() : 0u;
+  const int g = pair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  // This CTA's partial slots (stream-K) and the stride between the CTAs of
+  // consecutive work units that contribute to one of its tiles.
+  const int P = pair ? 2 : 1;
   // Let the next kernel in the stream start launching: its CTAs take SMs as
   // this grid's CTAs exit and wait (griddepcontrol.wait) before reading
   // anything this grid writes.
   ptx::griddep_launch_dependents();
   const int b0 = p.cta_start[g];
   const int b1 = p.cta_start[g + 1];
+  const bool in_cluster = p.cluster > 1 || pair;  // launched as clusters (uses the cluster barrier)
 
   if (warp >= 2 && warp <= 5) {
     // The epilogue warps are idle during set-up: they touch the whole
@@ -263,10 +284,14 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(ptx::smem_addr(&bars->acc_full[a]), 1);
-      ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), 128);
+      // pair mode: the even CTA's accumulator is free once both epilogues have
+      // read their halves (the odd CTA's epilogue arrives once, remotely)
+      ptx::mbar_init(ptx::smem_addr(&bars->acc_empty[a]), pair ? 129 : 128);
     }
     ptx::mbar_init(ptx::smem_addr(&bars->peer_done), 1);
     ptx::mbar_init(ptx::smem_addr(&bars->ack), 1);
+    if (pair)
+      for (int s = 0; s < p.stages; ++s) ptx::mbar_init(ptx::smem_addr(&bars->peer_full[s]), 1);
     if (p.cluster > 1 && ptx::cluster_ctarank() == 0) {
       // Rank 0 expects every peer's partial of its tile (whole 16-token
       // chunks up to the valid tokens) as one bulk copy per peer. This precedes
@@ -283,8 +308,13 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), p.tmem_cols);
-    ptx::tmem_relinquish();
+    if constexpr (pair) {
+      ptx::tmem_alloc_pair(ptx::smem_addr(&bars->tmem_base), p.tmem_cols);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(ptx::smem_addr(&bars->tmem_base), p.tmem_cols);
+      ptx::tmem_relinquish();
+    }
   }
   // Set-up barriers: the producers only need the mbarriers, so warp 0 (which
   // initialised them) releases the second producer warp (named barrier 2)
@@ -293,7 +323,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   // the cluster barrier once here; a peer waits on it before its first store
   // into rank 0.
   auto setup_wait = [&]() -> uint32_t {
-    if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+    if (in_cluster) ptx::cluster_arrive_relaxed();
     ptx::tc_fence_before();
     ptx::named_bar_sync(3, kGemmThreads);
     ptx::tc_fence_after();
@@ -332,12 +362,14 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     // one after another, so these small copies (the MMA needs them, and they
     // wait for the previous grid) do not queue behind the weight copies.
     ptx::named_bar_sync(2, bar2_threads);  // the barriers are initialised
-    if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+    if (in_cluster) ptx::cluster_arrive_relaxed();
     test_gate_wait();
     if (lane == 0 && !*abort_flag) {
       ptx::griddep_wait();  // X may be written by the previous grid
       const uint64_t pol_x = ptx::policy_evict_last();
-      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;       // smem bytes of a K-atom
+      // Pair mode: each CTA of the pair holds half of the token tile's rows.
+      const int xrows = pair ? p.npad / 2 : p.npad;
+      const uint32_t box = static_cast<uint32_t>(xrows) * 128u;        // smem bytes of a K-atom
       const uint32_t xb = static_cast<uint32_t>(p.box_rows) * 128u;    // bytes of one TMA box
       BlockWalker cx(units, p);
       Ring ring(static_cast<uint32_t>(p.stages));
@@ -347,7 +379,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
                                        SPENSE_DEVICE_TIMEOUT_PRODUCER, abort_flag))
           break;
         const GemmMember& mb = p.mem[cx.member];
-        const int y0 = cx.m_tile * p.npad;
+        const int y0 = cx.m_tile * p.npad + static_cast<int>(prank) * xrows;
         const uint32_t b_s = smem_base + ring.s * p.stage_bytes + kBlockBytes;
         const uint32_t full = ptx::smem_addr(&bars->full[ring.s]);
         if (cx.j < mb.nsb) {
@@ -371,18 +403,20 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     // the two issue streams concurrently.
     if (warp == 0) {
       __syncwarp();  // lane 0 initialised the barriers
-      if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+      if (in_cluster) ptx::cluster_arrive_relaxed();
       ptx::named_bar_arrive(3, kGemmThreads);
       if (bar2_threads > 32u) ptx::named_bar_arrive(2, bar2_threads);
     } else {
       ptx::named_bar_sync(2, bar2_threads);
-      if (p.cluster > 1) ptx::cluster_arrive_relaxed();
+      if (in_cluster) ptx::cluster_arrive_relaxed();
     }
     test_gate_wait();
     if (lane == 0 && !*abort_flag) {
       const int np = p.producers;
       const int me = warp == 0 ? 0 : 1;
-      const uint64_t pol_w = ptx::policy_evict_first();
+      // Weights stream once (evict first), unless neighbouring token tiles
+      // re-read them (then they stay in L2 for the second read).
+      const uint64_t pol_w = p.w_keep ? ptx::policy_evict_normal() : ptx::policy_evict_first();
       const uint64_t pol_x = ptx::policy_evict_last();
       const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;         // smem bytes of a K-atom
       // bytes one TMA box of activations loads (none here when the activation loader issues them)
@@ -394,15 +428,16 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         const uint32_t a_s = smem_base + s * p.stage_bytes;
         const uint32_t full = ptx::smem_addr(&bars->full[s]);
         const uint32_t piece = kBlockBytes / static_cast<uint32_t>(p.bulk_split);
+        const int wt = c.weight_tile(p, prank);
         if (c.j < mb.nsb) {
-          const size_t blk = static_cast<size_t>(c.local_tile) * mb.nsb + c.j;
+          const size_t blk = static_cast<size_t>(wt) * mb.nsb + c.j;
           ptx::mbar_arrive_expect_tx(full, kBlockBytes + kMetaBlockBytes + 2 * xbytes);
           for (int q = 0; q < p.bulk_split; ++q)
             ptx::bulk_g2s(a_s + q * piece, mb.vs_t + blk * kBlockBytes + q * piece, piece, full, pol_w);
           ptx::bulk_g2s(a_s + kBlockBytes + p.b_bytes, mb.e_t + blk * kMetaBlockBytes, kMetaBlockBytes,
                         full, pol_w);
         } else {
-          const size_t blk = static_cast<size_t>(c.local_tile) * mb.ndb + (c.j - mb.nsb);
+          const size_t blk = static_cast<size_t>(wt) * mb.ndb + (c.j - mb.nsb);
           ptx::mbar_arrive_expect_tx(full, kBlockBytes + xbytes);
           for (int q = 0; q < p.bulk_split; ++q)
             ptx::bulk_g2s(a_s + q * piece, mb.wd_t + blk * kBlockBytes + q * piece, piece, full, pol_w);
@@ -432,12 +467,13 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         for (int i = pre; i < last; ++i, cp.advance(p)) {
           if (i % np != me) continue;
           const GemmMember& mb = p.mem[cp.member];
+          const int wt = cp.weight_tile(p, prank);
           if (cp.j < mb.nsb) {
-            const size_t blk = static_cast<size_t>(cp.local_tile) * mb.nsb + cp.j;
+            const size_t blk = static_cast<size_t>(wt) * mb.nsb + cp.j;
             ptx::prefetch_l2_bulk(mb.vs_t + blk * kBlockBytes, kBlockBytes);
             ptx::prefetch_l2_bulk(mb.e_t + blk * kMetaBlockBytes, kMetaBlockBytes);
           } else {
-            const size_t blk = static_cast<size_t>(cp.local_tile) * mb.ndb + (cp.j - mb.nsb);
+            const size_t blk = static_cast<size_t>(wt) * mb.ndb + (cp.j - mb.nsb);
             ptx::prefetch_l2_bulk(mb.wd_t + blk * kBlockBytes, kBlockBytes);
           }
         }
@@ -462,21 +498,45 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     const uint32_t tmem_base = setup_wait();
-    if (lane == 0) {
-      const uint32_t idesc_sp = ptx::idesc_f8(static_cast<uint32_t>(p.npad), true);
-      const uint32_t idesc_d = ptx::idesc_f8(static_cast<uint32_t>(p.npad), false);
+    // Pair mode: before the first signal into the other CTA of the pair, its
+    // barriers must be initialised (it arrived on the cluster barrier after).
+    if (pair) ptx::cluster_wait();
+    if (lane == 0 && pair && prank == 1) {
+      // Odd CTA of a pair: relay. Its stages land on its own barriers; the
+      // even CTA issues the pair's MMAs once both halves of a stage are in,
+      // so each landed stage is announced to it.
+      Ring ring(static_cast<uint32_t>(p.stages));
+      const uint32_t peer_full0 = ptx::mapa(ptx::smem_addr(&bars->peer_full[0]), 0u);
+      for (int i = 0; i < b1 - b0; ++i, ring.advance()) {
+        if (!wait_bar(ptx::smem_addr(&bars->full[ring.s]), ring.ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
+                      abort_flag))
+          break;
+        ptx::mbar_arrive_remote_release(peer_full0 + 8u * ring.s);
+      }
+    } else if (lane == 0) {
+      const uint32_t mma_m = pair ? 256u : 128u;
+      const uint32_t idesc_sp = ptx::idesc_f8(static_cast<uint32_t>(p.npad), true, mma_m);
+      const uint32_t idesc_d = ptx::idesc_f8(static_cast<uint32_t>(p.npad), false, mma_m);
       const uint32_t e_col0 = static_cast<uint32_t>(p.nacc * p.npad);
-      const uint32_t box = static_cast<uint32_t>(p.npad) * 128u;
+      const uint32_t box = static_cast<uint32_t>(pair ? p.npad / 2 : p.npad) * 128u;
       Ring ring(static_cast<uint32_t>(p.stages));
       uint32_t ebuf = 0;
       bool ok = true;
+      // Completion signals: to this CTA, or in pair mode to both CTAs' barriers.
+      auto commit = [&](uint32_t bar) {
+        if constexpr (pair)
+          ptx::mma_commit_pair(bar, 0x3);
+        else
+          ptx::mma_commit(bar);
+      };
       for (int u = 0; ok && u < units.count; ++u) {
         int t, j0, j1;
         units.get(u, t, j0, j1);
         const uint32_t acc = static_cast<uint32_t>(u % p.nacc);
         const uint32_t aph = static_cast<uint32_t>((u / p.nacc) & 1);
-        if (!wait_bar(ptx::smem_addr(&bars->acc_empty[acc]), aph ^ 1u, p.status,
-                      SPENSE_DEVICE_TIMEOUT_MMA, abort_flag)) {
+        const uint32_t acc_bar = ptx::smem_addr(&bars->acc_empty[acc]);
+        if (!(pair ? wait_bar_cluster(acc_bar, aph ^ 1u, p.status, SPENSE_DEVICE_TIMEOUT_MMA, abort_flag)
+                   : wait_bar(acc_bar, aph ^ 1u, p.status, SPENSE_DEVICE_TIMEOUT_MMA, abort_flag))) {
           ok = false;
           break;
         }
@@ -485,7 +545,9 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         const int nsb_u = p.mem[member_of(p, t / p.m_tiles)].nsb;  // 2:4 blocks of this tile
         for (int j = j0; j < j1; ++j, ring.advance()) {
           if (!wait_bar(ptx::smem_addr(&bars->full[ring.s]), ring.ph, p.status, SPENSE_DEVICE_TIMEOUT_MMA,
-                        abort_flag)) {
+                        abort_flag) ||
+              (pair && !wait_bar_cluster(ptx::smem_addr(&bars->peer_full[ring.s]), ring.ph, p.status,
+                                         SPENSE_DEVICE_TIMEOUT_MMA, abort_flag))) {
             ok = false;
             break;
           }
@@ -495,13 +557,22 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
           const uint32_t e_s = b_s + p.b_bytes;
           if (j < nsb_u) {
             const uint32_t e_tmem = tmem_base + e_col0 + ebuf * 8u;
-            ptx::tmem_cp_128x128b(e_tmem, ptx::desc_rows16(e_s));
-            ptx::tmem_cp_128x128b(e_tmem + 4u, ptx::desc_rows16(e_s + 2048u));
+            if constexpr (pair) {
+              ptx::tmem_cp_128x128b_pair(e_tmem, ptx::desc_rows16(e_s));
+              ptx::tmem_cp_128x128b_pair(e_tmem + 4u, ptx::desc_rows16(e_s + 2048u));
+            } else {
+              ptx::tmem_cp_128x128b(e_tmem, ptx::desc_rows16(e_s));
+              ptx::tmem_cp_128x128b(e_tmem + 4u, ptx::desc_rows16(e_s + 2048u));
+            }
 #pragma unroll
             for (uint32_t k = 0; k < 4; ++k) {
               const uint64_t ad = ptx::desc_sw128(a_s + 32u * k);
               const uint64_t bd = ptx::desc_sw128(b_s + (k >> 1) * box + (k & 1u) * 64u);
-              ptx::mma_sp_f8(d_tmem, ad, bd, e_tmem + 2u * k, idesc_sp, (j > j0 || k > 0) ? 1u : 0u);
+              const uint32_t accum = (j > j0 || k > 0) ? 1u : 0u;
+              if constexpr (pair)
+                ptx::mma_sp_f8_pair(d_tmem, ad, bd, e_tmem + 2u * k, idesc_sp, accum);
+              else
+                ptx::mma_sp_f8(d_tmem, ad, bd, e_tmem + 2u * k, idesc_sp, accum);
             }
             ebuf ^= 1u;
           } else {
@@ -509,13 +580,17 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             for (uint32_t k = 0; k < 4; ++k) {
               const uint64_t ad = ptx::desc_sw128(a_s + 32u * k);
               const uint64_t bd = ptx::desc_sw128(b_s + 32u * k);
-              ptx::mma_f8(d_tmem, ad, bd, idesc_d, (j > j0 || k > 0) ? 1u : 0u);
+              const uint32_t accum = (j > j0 || k > 0) ? 1u : 0u;
+              if constexpr (pair)
+                ptx::mma_f8_pair(d_tmem, ad, bd, idesc_d, accum);
+              else
+                ptx::mma_f8(d_tmem, ad, bd, idesc_d, accum);
             }
           }
-          ptx::mma_commit(ptx::smem_addr(&bars->empty[ring.s]));
+          commit(ptx::smem_addr(&bars->empty[ring.s]));
         }
         if (!ok) break;
-        ptx::mma_commit(ptx::smem_addr(&bars->acc_full[acc]));
+        commit(ptx::smem_addr(&bars->acc_full[acc]));
       }
       if (ok && p.cluster > 1 && ptx::cluster_ctarank() == 0 &&
           wait_bar_cluster(ptx::smem_addr(&bars->peer_done), 0, p.status, SPENSE_DEVICE_TIMEOUT_EPILOGUE,
@@ -555,7 +630,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       stage_sx(m0);
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
-      const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+      const int n = (P * (n_tile - mb.tile_begin) + static_cast<int>(prank)) * kTileRows + row;
       const bool row_ok = n < mb.N;
       const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
       int nb_t;
@@ -563,11 +638,13 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       const int g_lo = block_owner(p, tb);
       const int g_hi = block_owner(p, tb + nb_t - 1);
       const int lo_slot = (p.cta_start[g_lo] >= tb) ? 0 : 1;
-      const float* lo_part =
-          p.partials + (static_cast<size_t>(g_lo) * 2 + lo_slot) * slot_elems + static_cast<size_t>(row) * p.npad;
-      const float* next_part =
-          p.partials + (static_cast<size_t>(g_lo + 1) * 2) * slot_elems + static_cast<size_t>(row) * p.npad;
-      const size_t stride = 2 * slot_elems;  // from contributor gg to gg + 1 (slot 0)
+      // The contributors' partials of this CTA's rows: work unit gg's CTA of
+      // the same rank in the pair (CTA gg x P + rank).
+      const float* lo_part = p.partials + (static_cast<size_t>(g_lo * P + prank) * 2 + lo_slot) * slot_elems +
+                             static_cast<size_t>(row) * p.npad;
+      const float* next_part = p.partials + (static_cast<size_t>((g_lo + 1) * P + prank) * 2) * slot_elems +
+                               static_cast<size_t>(row) * p.npad;
+      const size_t stride = static_cast<size_t>(2 * P) * slot_elems;  // from contributor gg to gg + 1 (slot 0)
       const int others = g_hi - g_lo;
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
         const int nq = min(4, (m_valid - c0 + 3) >> 2);  // float4 groups holding valid tokens
@@ -615,7 +692,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
           }
         }
       }
-      if (et == 0) p.counters[t] = 0u;  // re-arm for the next launch (ordered by the kernel boundary)
+      if (et == 0) p.counters[t * P + prank] = 0u;  // re-arm for the next launch (ordered by the kernel boundary)
     };
 
     // Tiles this CTA must finish. Their fix-ups wait until this CTA has
@@ -746,7 +823,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       const int m0 = (t - n_tile * p.m_tiles) * p.npad;
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
-      const int n = (n_tile - mb.tile_begin) * kTileRows + row;
+      const int n = (P * (n_tile - mb.tile_begin) + static_cast<int>(prank)) * kTileRows + row;
       const bool row_ok = n < mb.N;
       int nb_t;
       const int tb = tile_block0(p, t, &nb_t);
@@ -764,7 +841,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       float* part = nullptr;
       if (!whole) {
         const int slot = (b0 >= tb) ? 0 : 1;
-        part = p.partials + (static_cast<size_t>(g) * 2 + slot) * slot_elems + static_cast<size_t>(row) * p.npad;
+        part = p.partials + (static_cast<size_t>(g * P + prank) * 2 + slot) * slot_elems +
+               static_cast<size_t>(row) * p.npad;
       }
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
         uint32_t v[16];
@@ -789,7 +867,14 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         }
       }
       ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
+      if (pair && prank == 1) {
+        // The pair's accumulator barrier lives in the even CTA: one arrival
+        // there once all 128 threads of this CTA have read their rows.
+        ptx::named_bar_sync(1, 128);
+        if (et == 0) ptx::mbar_arrive_remote_release(ptx::mapa(ptx::smem_addr(&bars->acc_empty[acc]), 0u));
+      } else {
+        ptx::mbar_arrive(ptx::smem_addr(&bars->acc_empty[acc]));
+      }
       if (!whole) {
         // Publish this CTA's partial: the named barrier orders the 128 threads'
         // stores before thread 0's release-acquire ticket at GPU scope.
@@ -797,7 +882,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         if (et == 0) {
           const int g_lo = block_owner(p, tb);
           const int g_hi = block_owner(p, tb + nb_t - 1);
-          const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t, 1u);
+          const unsigned int old = ptx::atom_add_acq_rel_gpu(p.counters + t * P + prank, 1u);
           bars->fix_flag = (old == static_cast<unsigned int>(g_hi - g_lo)) ? 1 : 0;
         }
         ptx::named_bar_sync(1, 128);
@@ -819,6 +904,19 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   }
 
   __syncwarp();
+  if (pair && prank == 1 && warp == 0 && lane == 0) {
+    // The even CTA's completion signals land in this CTA's stage barriers
+    // asynchronously: wait (bounded) for the last one of every stage before
+    // this CTA may exit. After a failure they may never come; the wait runs out.
+    const int nb = b1 - b0;
+    const uint64_t t0 = ptx::globaltimer();
+    for (int i = nb > p.stages ? nb - p.stages : 0; i < nb; ++i) {
+      const uint32_t bar = ptx::smem_addr(&bars->empty[i % p.stages]);
+      const uint32_t parity = static_cast<uint32_t>((i / p.stages) & 1);
+      while (!ptx::mbar_try_wait(bar, parity) && ptx::globaltimer() - t0 < kWaitLimitNs) {
+      }
+    }
+  }
   ptx::tc_fence_before();
   __syncthreads();
   // Tensor memory is released before any cluster-barrier operation: a
@@ -826,7 +924,18 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
   // keeping the CTA (and its SM slot) alive.
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(bars->tmem_base, p.tmem_cols);
+    if constexpr (pair)
+      ptx::tmem_dealloc_pair(bars->tmem_base, p.tmem_cols);
+    else
+      ptx::tmem_dealloc(bars->tmem_base, p.tmem_cols);
+  }
+  if (pair) {
+    // Neither CTA of a pair leaves while the other may still signal into it:
+    // every thread has arrived on the cluster barrier once at set-up (only the
+    // MMA warp waited on that phase); all wait for it, then meet once more.
+    if (warp != 1) ptx::cluster_wait();
+    ptx::cluster_arrive();
+    ptx::cluster_wait();
   }
   if (p.cluster > 1) {
     if (ptx::cluster_ctarank() != 0) {
@@ -868,8 +977,11 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
   cudaError_t st = cudaGetDevice(&dev);
   if (st != cudaSuccess) return st;
   if (configured_for != dev) {
-    st = cudaFuncSetAttribute(spense_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    st = cudaFuncSetAttribute(spense_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(gemm_max_smem()));
+    if (st == cudaSuccess)
+      st = cudaFuncSetAttribute(spense_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(gemm_max_smem()));
     if (st != cudaSuccess) return st;
     configured_for = dev;
   }
@@ -881,7 +993,7 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
     return !(e != nullptr && e[0] == '0');
   }();
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned int>(p.grid));
+  cfg.gridDim = dim3(static_cast<unsigned int>(p.grid * (p.pair ? 2 : 1)));
   cfg.blockDim = dim3(kGemmThreads + 32 * (p.producers - 1) + 32 * p.x_warp);
   cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = stream;
@@ -889,14 +1001,15 @@ cudaError_t launch_gemm(const CUtensorMap& tmap_x, const GemmParams& p, uint32_t
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = static_cast<unsigned int>(p.cluster > 1 ? p.cluster : 1);
+  attr[1].val.clusterDim.x = static_cast<unsigned int>(p.pair ? 2 : (p.cluster > 1 ? p.cluster : 1));
   attr[1].val.clusterDim.y = 1;
   attr[1].val.clusterDim.z = 1;
   attr[2].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
   attr[2].val.clusterSchedulingPolicyPreference = cluster_policy();
   cfg.attrs = attr;
-  cfg.numAttrs = p.cluster > 1 ? 3 : 2;
-  return cudaLaunchKernelEx(&cfg, spense_gemm_kernel, tmap_x, p);
+  cfg.numAttrs = (p.cluster > 1 || p.pair) ? 3 : 2;
+  return p.pair ? cudaLaunchKernelEx(&cfg, spense_gemm_kernel<true>, tmap_x, p)
+                : cudaLaunchKernelEx(&cfg, spense_gemm_kernel<false>, tmap_x, p);
 }
 
 }  // namespace spense

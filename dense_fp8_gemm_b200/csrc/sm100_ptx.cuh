@@ -56,6 +56,12 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+__device__ __forceinline__ uint64_t policy_evict_normal() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -103,6 +109,25 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// Tensor memory of a CTA pair (tcgen05 cta_group::2): one warp of each CTA of
+// the pair (the same warp index in both) issues these together; the pair gets
+// the same columns in both CTAs, and the address is written to the same
+// shared-memory offset in both.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -133,6 +158,48 @@ __device__ __forceinline__ void mma_sp_f8(uint32_t d_tmem, uint64_t a_desc, uint
       "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Pair forms (cta_group::2), issued by one thread of the pair's even CTA: the
+// MMA is M = 256; rows 0-127 of A come from the even CTA's shared memory,
+// rows 128-255 from the odd CTA's (the same offset), each CTA holds half of
+// B's N rows at the same offset, and each CTA's tensor memory receives its
+// 128 rows x N of D (and, for .sp, reads its own rows' metadata).
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_sp_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the mbarrier at offset `bar` in every CTA of `cta_mask`
+// when every tcgen05 operation of the pair this thread issued so far has
+// completed (the pair's completion signal).
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// tcgen05.cp of the pair: 128 rows x 16 bytes from each CTA's shared memory
+// (the same offset) into that CTA's tensor memory.
+__device__ __forceinline__ void tmem_cp_128x128b_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued so far
@@ -220,6 +287,13 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
   return r;
 }
 
+// Arrive on an mbarrier of another CTA of the cluster, releasing this
+// thread's prior memory accesses (and those ordered before them) at cluster
+// scope; pairs with mbar_try_wait_cluster.
+__device__ __forceinline__ void mbar_arrive_remote_release(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster without ordering any
 // memory access (a pure signal).
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
@@ -282,6 +356,12 @@ __device__ __forceinline__ void st_smem_v4(uint32_t saddr, float4 v) {
                : "memory");
 }
 
+// Arrive on the cluster barrier without waiting, releasing this thread's
+// earlier memory accesses at cluster scope.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
 // Arrive on the cluster barrier without waiting and without ordering any
 // earlier memory access.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
@@ -309,12 +389,13 @@ __device__ __forceinline__ uint64_t desc_rows16(uint32_t saddr) {
          (1ull << 46);
 }
 
-// Instruction descriptor: e4m3 x e4m3 -> f32, both K-major, M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_f8(uint32_t n, bool sparse) {
+// Instruction descriptor: e4m3 x e4m3 -> f32, both K-major, M = m (128, or
+// 256 for a CTA pair), N = n.
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t n, bool sparse, uint32_t m = 128u) {
   return (1u << 4)                    // D format f32
          | (0u << 7) | (0u << 10)     // A, B e4m3
          | ((n >> 3) << 17)           // N / 8
-         | ((128u >> 4) << 24)        // M / 16
+         | ((m >> 4) << 24)           // M / 16
          | (sparse ? (1u << 2) : 0u); // sparse flag
 }
 

@@ -191,6 +191,32 @@ int cluster_mode() {
   return v;
 }
 
+// SPENSE_W_KEEP: -1 (default) = automatic (weights keep the evict-normal L2
+// policy when several token tiles re-read them: down 5120x27648 at 256 tokens
+// 65.2 -> 63.9 us), 0 = always stream them evict-first, 1 = always keep.
+int w_keep_knob() {
+  static const int v = env_int("SPENSE_W_KEEP", -1, -1, 1);
+  return v;
+}
+
+// SPENSE_PAIR: 0 (default) = never use CTA pairs; 1 = pairs for more than 64
+// tokens; 2 = pairs whenever the layout allows. Pairs are correct but were
+// measured slower than single CTAs on every shape of the workloads (gate+up
+// 55296x5120 at 256 tokens 121 vs 95 us, at 64 tokens 70 vs 40 us): with 256
+// tokens only one accumulator fits in tensor memory, so each tile's epilogue
+// stalls the MMAs, and at 64 tokens the halved activation boxes (4 KiB) keep
+// many small copies in flight (5.5 us from issue to landing vs 1.5 us).
+int pair_knob() {
+  static const int v = env_int("SPENSE_PAIR", 0, 0, 2);
+  return v;
+}
+
+// SPENSE_PAIRS_MAX: at most this many CTA pairs per launch (0 = automatic).
+int pairs_max_knob() {
+  static const int v = env_int("SPENSE_PAIRS_MAX", 0, 0, kMaxGrid);
+  return v;
+}
+
 int bulk_split() {
   static const int v = [] {
     const int x = env_int("SPENSE_BULK_SPLIT", 1, 1, 4);
@@ -225,10 +251,20 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // which halves the repeat reads and gives each CTA longer whole tiles.
   const long long tiles64 = row_tiles * ((M + 63) / 64);
   const bool small_weight = weight_units * 4096ll <= (32ll << 20);  // cost units are 4 KiB
-  const int T = token_tile_knob() != 0 ? token_tile_knob()
-                                       : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128);
+  // Pair mode (opt-in, see pair_knob): two CTAs on two SMs share one MMA of
+  // 256 weight rows (tcgen05 cta_group::2), each holding half of the token
+  // tile, so every activation byte staged in shared memory serves twice the
+  // weight rows, and token tiles of up to 256 tokens read each weight once.
+  const int pk = pair_knob();
+  pl.pair = (x_warp() && (pk == 2 || (pk == 1 && M > 64))) ? 1 : 0;
+  const int T = token_tile_knob() != 0
+                    ? token_tile_knob()
+                    : (pl.pair ? kMaxTokenTile
+                               : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128));
   pl.npad = M > T ? T : static_cast<int>(round_up(static_cast<size_t>(M), 16));
-  pl.box_rows = static_cast<int>(M > T ? T : M);
+  // rows one activation box loads: the valid rows of the token tile, or in
+  // pair mode this CTA's half of it (rows past M read as zeros)
+  pl.box_rows = pl.pair ? pl.npad / 2 : static_cast<int>(M > T ? T : M);
   pl.m_tiles = static_cast<int>((M + T - 1) / T);
   pl.count = count;
   long long n_tiles = 0, blocks = 0, cost = 0;
@@ -240,16 +276,18 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
       return fail(SPENSE_ERR_ARG,
                   "packed weights sharing a launch need the same device, K and column order of X (the same "
                   "scattered dense set, or none)");
-    pl.mem_tiles[i] = h->n_tiles;
+    // work tiles of member i: its 128-row tiles, or in pair mode pairs of them
+    const int ut = pl.pair ? (h->n_tiles + 1) / 2 : h->n_tiles;
+    pl.mem_tiles[i] = ut;
     pl.mem_nsb[i] = h->nsb;
     pl.mem_ndb[i] = h->ndb;
     pl.mem_cost[i] = kCostSparse * h->nsb + kCostDense * h->ndb;
     pl.mem_block_begin[i] = static_cast<int>(std::min<long long>(blocks, 1ll << 31));
     pl.mem_cost_begin[i] = cost;
-    const long long tiles_i = static_cast<long long>(h->n_tiles) * pl.m_tiles;
+    const long long tiles_i = static_cast<long long>(ut) * pl.m_tiles;
     blocks += tiles_i * (h->nsb + h->ndb);
     cost += tiles_i * pl.mem_cost[i];
-    n_tiles += h->n_tiles;
+    n_tiles += ut;
     pl.min_tile_cost = std::min(pl.min_tile_cost, pl.mem_cost[i]);
     pl.any_sparse = pl.any_sparse || h->nsb > 0;
   }
@@ -264,7 +302,7 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   long long grid = pl.total_cost / std::max<long long>(kCostSparse, min_cta_weight());
   pl.bulk_split = bulk_split();
   pl.producers = producers();
-  pl.b_bytes = static_cast<uint32_t>(pl.npad) * (pl.any_sparse ? 256u : 128u);
+  pl.b_bytes = static_cast<uint32_t>(pl.pair ? pl.npad / 2 : pl.npad) * (pl.any_sparse ? 256u : 128u);
   pl.stage_bytes = kBlockBytes + pl.b_bytes + (pl.any_sparse ? kMetaBlockBytes : 0);
   const uint32_t reserve = 1024 + kBarrierBytes;  // alignment slack + barrier area
   // Ring and TMEM for `cps` CTAs per SM; false if two stages or the
@@ -280,6 +318,8 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
     return *cols <= tmem_budget;
   };
   auto slots_for = [&](int cps) {
+    if (pl.pair)  // one pair per two SMs
+      return std::min<long long>(pairs_max_knob() > 0 ? pairs_max_knob() : sms / 2, kMaxGrid);
     return std::min<long long>(static_cast<long long>(sms) * std::min(cps, grid_per_sm()), kMaxGrid);
   };
   // Few tiles (at most half the CTA slots): the CTAs of a cluster of S split
@@ -313,10 +353,16 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // other count takes the other.
   const int knob = ctas_per_sm_knob();
   int cps = knob != 0 ? knob : ((pl.tiles > 2 * sms || pl.npad > 32) ? 1 : 2);
-  pl.cluster = cluster_for(cps);
-  if (pl.cluster == 1 && knob == 0 && cluster_for(3 - cps) > 1) {
-    cps = 3 - cps;
+  if (pl.pair) {
+    // pairs: one CTA per SM with the whole ring, stream-K over pair tiles
+    cps = 1;
+    pl.cluster = 1;
+  } else {
     pl.cluster = cluster_for(cps);
+    if (pl.cluster == 1 && knob == 0 && cluster_for(3 - cps) > 1) {
+      cps = 3 - cps;
+      pl.cluster = cluster_for(cps);
+    }
   }
   pl.recv_bytes = pl.cluster > 1 ? static_cast<uint32_t>(pl.cluster - 1) * kTileRows * pl.npad * 4u : 0u;
   if (!fit_ring(cps, pl.recv_bytes, &pl.stages, &pl.nacc, &pl.tmem_cols)) {
@@ -383,11 +429,14 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   WorkspaceLayout& w = pl.ws;
   size_t off = 256;  // header: status word
   w.counters_off = off;
-  w.counters_bytes = round_up(static_cast<size_t>(pl.tiles) * 4, 256);
+  const int ctas_per_unit = pl.pair ? 2 : 1;
+  // one arrival counter per CTA tile (in pair mode each CTA of a pair tile counts its own rows)
+  w.counters_bytes = round_up(static_cast<size_t>(pl.tiles) * ctas_per_unit * 4, 256);
   off += w.counters_bytes;
   w.partials_off = off;
   // fp32 partials of shared tiles: stream-K only (a cluster reduces in shared memory)
-  w.partials_bytes = pl.cluster > 1 ? 0 : static_cast<size_t>(pl.grid) * 2 * pl.npad * kTileRows * 4;
+  w.partials_bytes =
+      pl.cluster > 1 ? 0 : static_cast<size_t>(pl.grid) * ctas_per_unit * 2 * pl.npad * kTileRows * 4;
   off += w.partials_bytes;
   w.xg_off = off;
   w.xg_bytes = h0->perm ? round_up(static_cast<size_t>(M * h0->K), 256) : 0;
@@ -477,7 +526,8 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
     m.Ks = static_cast<int>(hs[i]->Ks);
     m.block_begin = pl.mem_block_begin[i];
     m.ldy = static_cast<int>(ldy != nullptr ? ldy[i] : hs[i]->N);
-    tile_begin += hs[i]->n_tiles;
+    m.row_tiles = hs[i]->n_tiles;
+    tile_begin += pl.mem_tiles[i];
   }
   p.n_members = count;
   p.s_x = x_scale;
@@ -502,6 +552,8 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
   p.recv_bytes = pl.recv_bytes;
   p.l2_prefetch = l2_prefetch_for(pl);
   p.x_warp = x_warp();
+  p.w_keep = w_keep_knob() >= 0 ? w_keep_knob() : (pl.m_tiles > 1 ? 1 : 0);
+  p.pair = pl.pair;
 #ifdef SPENSE_TEST_HOOKS
   // Test build only: with SPENSE_TEST_STALL=1 the loaders wait on header word
   // 16 of the workspace, which nothing sets, so every launch ends by timeout.
@@ -934,6 +986,7 @@ spense_status spense_plan_shapes(int count, const int64_t* N, const int64_t* K, 
   out->stage_bytes = pl.stage_bytes;
   out->recv_bytes = pl.recv_bytes;
   out->l2_prefetch = l2_prefetch_for(pl);
+  out->pair = pl.pair;
   out->total_blocks = pl.cta_start[pl.grid];
   out->workspace_bytes = pl.ws.total_device;
   for (int g = 0; g <= pl.grid; ++g) out->cta_start[g] = pl.cta_start[g];

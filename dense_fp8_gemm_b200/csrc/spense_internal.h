@@ -34,7 +34,7 @@ struct WorkspaceLayout {
 };
 
 constexpr int kMaxGroup = 4;    // weight matrices sharing one activation tensor in one launch
-constexpr int kMaxGrid = 320;   // CTAs per launch (up to two per SM)
+constexpr int kMaxGrid = 320;   // work units per launch (CTAs, up to two per SM; or CTA pairs)
 
 struct GemmPlan {
   int npad;        // MMA N (tokens per tile, multiple of 16)
@@ -63,7 +63,8 @@ struct GemmPlan {
   int producers;
   int cluster;
   uint32_t recv_bytes;
-  int cta_start[kMaxGrid + 1];  // first linear block of each CTA; [grid] = total blocks
+  int pair;        // 1: CTA pairs (tcgen05 cta_group::2) share 256-row MMAs; the work units are pairs
+  int cta_start[kMaxGrid + 1];  // first linear block of each work unit (CTA, or pair); [grid] = total blocks
   WorkspaceLayout ws;
 };
 
@@ -82,6 +83,7 @@ struct GemmMember {
   int Ks;            // X column where the dense region starts
   int block_begin;   // first linear block of the member's tiles
   int ldy;           // output row stride in elements (>= N)
+  int row_tiles;     // 128-row tiles of the member (pair mode: its tiles above count pairs of them)
 };
 
 struct GemmParams {
@@ -104,6 +106,8 @@ struct GemmParams {
   uint32_t recv_bytes;            // cluster mode: rank 0's receive area for the peers' partials
   int l2_prefetch;                // blocks past the first ring's worth prefetched into L2 at start
   int x_warp;                     // 1: a warp of its own issues the activation-tile loads
+  int w_keep;                     // 1: weight copies use the evict-normal L2 policy (re-read by token tiles)
+  int pair;                       // 1: pair mode (grid = 2 CTAs per work unit, cluster of 2, M = 256 MMAs)
 };
 
 // Kernels (defined in the .cu files).

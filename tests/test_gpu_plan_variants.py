@@ -1,6 +1,6 @@
 """GPU parity of every launch plan the library can choose, not only the
 default one. The plan knobs (token tile, CTAs per SM, cluster split or
-stream-K, loader warps, bulk-copy split, programmatic dependent launch) are
+stream-K, CTA pairs, loader warps, bulk-copy split, programmatic dependent launch) are
 read once per process, so each variant runs in a child process that packs a
 few weights, runs the GEMM (single and grouped launches, ragged token counts,
 tail and scattered dense sets) and checks every output against the oracle
@@ -68,6 +68,8 @@ VARIANTS = [
     {"SPENSE_TOKEN_TILE": "256"},
     {"SPENSE_PRODUCERS": "1", "SPENSE_BULK_SPLIT": "2"},
     {"SPENSE_PDL": "0", "SPENSE_GRID_PER_SM": "1"},
+    {"SPENSE_PAIR": "2"},                  # CTA pairs (tcgen05 cta_group::2) at every token count
+    {"SPENSE_PAIR": "1", "SPENSE_TOKEN_TILE": "128"},  # pairs above 64 tokens, two token tiles at 200
 ]
 
 

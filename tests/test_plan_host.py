@@ -1,9 +1,10 @@
 """Host-side checks of the launch planner (spense_plan_shapes, no GPU): for
 the workloads' shapes and token counts from 1 to 65535, every plan streams
-every weight block exactly once, keeps a cluster inside one tile, fits the
-shared-memory and tensor-memory budgets of its CTAs-per-SM choice, covers
-every token, and sizes its workspace for its partials; and the token-tile and
-cluster choices that the measurements justify are the ones made.
+every weight block exactly once (in pair mode once per CTA of a pair, whose
+work tiles are pairs of 128-row tiles), keeps a cluster inside one tile, fits
+the shared-memory and tensor-memory budgets of its CTAs-per-SM choice, covers
+every token, and sizes its workspace for its partials; and the token-tile,
+cluster and pair choices that the measurements justify are the ones made.
 """
 import pytest
 
@@ -43,16 +44,21 @@ def blocks_of(N, K, Kd):
 def test_plan_invariants(name, M):
     shapes = SHAPES[name]
     p = spense.plan_shapes(shapes, M, SMS)
-    cps, S, grid, npad = p["ctas_per_sm"], p["cluster"], p["grid"], p["npad"]
+    cps, S, grid, npad, pair = p["ctas_per_sm"], p["cluster"], p["grid"], p["npad"], p["pair"]
+    # pair mode (CTA pairs, 256-row MMAs) is opt-in: never chosen by default
+    assert pair == 0
     # tokens: tiles of npad (a multiple of 16) cover M, the last one not empty
     assert npad % 16 == 0 and 16 <= npad <= 256
     assert p["m_tiles"] * npad >= M > (p["m_tiles"] - 1) * npad
-    assert p["box_rows"] == min(M, npad)
-    # blocks: member by member, row tile by row tile, every token tile of a row tile
+    # activation boxes: the valid rows of a tile, or each CTA's half of it in pair mode
+    assert p["box_rows"] == (npad // 2 if pair else min(M, npad))
+    # blocks: member by member, work tile by work tile (a 128-row tile, or a pair of them), every
+    # token tile of a work tile
     total, tile_first = 0, []
     n_tiles = 0
     for N, K, Kd in shapes:
         nt, nsb, ndb = blocks_of(N, K, Kd)
+        nt = -(-nt // 2) if pair else nt
         n_tiles += nt
         for _ in range(nt * p["m_tiles"]):
             tile_first.append(total)
@@ -63,8 +69,10 @@ def test_plan_invariants(name, M):
     cs = p["cta_start"]
     assert cs[0] == 0 and cs[-1] == total and len(cs) == grid + 1
     assert all(a < b for a, b in zip(cs, cs[1:])), "a CTA with an empty or negative block range"
-    # grid and CTAs per SM
-    assert cps in (1, 2) and 1 <= grid <= min(spense.PLAN_MAX_GRID, SMS * cps)
+    # grid (work units: CTAs, or CTA pairs on two SMs each) and CTAs per SM
+    assert cps in (1, 2) and 1 <= grid <= min(spense.PLAN_MAX_GRID, SMS * cps // (2 if pair else 1))
+    if pair:
+        assert cps == 1 and S == 1
     # cluster split: S consecutive CTAs share exactly one tile's blocks
     assert S in (1, 2, 4, 8)
     if S > 1:
@@ -76,7 +84,8 @@ def test_plan_invariants(name, M):
         assert p["recv_bytes"] == 0
     # shared memory: the ring (at least two stages) plus the receive area within the CTA's share
     any_sparse = any(K - Kd > 0 for _, K, Kd in shapes)
-    assert p["stage_bytes"] == 16384 + npad * (256 if any_sparse else 128) + (4096 if any_sparse else 0)
+    xrows = npad // 2 if pair else npad  # token rows of a stage's activation tile in this CTA
+    assert p["stage_bytes"] == 16384 + xrows * (256 if any_sparse else 128) + (4096 if any_sparse else 0)
     assert p["stages"] >= 2
     assert p["smem_bytes"] == RESERVE + p["stages"] * p["stage_bytes"] + p["recv_bytes"]
     assert p["smem_bytes"] <= SMEM_MAX // cps - (1024 if cps > 1 else 0)
@@ -85,23 +94,23 @@ def test_plan_invariants(name, M):
     assert p["nacc"] * npad + 16 <= p["tmem_cols"] <= 512 // cps
     # stream-K: the workspace holds every CTA's two fp32 partial slots (a cluster reduces in shared memory)
     if S == 1:
-        assert p["workspace_bytes"] >= grid * 2 * npad * 128 * 4
+        assert p["workspace_bytes"] >= grid * (2 if pair else 1) * 2 * npad * 128 * 4
     assert p["l2_prefetch"] == (4 if S > 1 else 0)
 
 
-@pytest.mark.parametrize("name,M,npad,S,cps", [
-    ("qkv", 16, 16, 2, 2),      # the decode bench launch: clusters of 2, two CTAs per SM
-    ("o", 16, 16, 4, 2),        # o_proj: clusters of 4
-    ("q", 64, 64, 2, 1),
-    ("q", 128, 64, 2, 2),       # 128 tiles of 64 tokens: clusters only with two CTAs per SM
-    ("gateup", 16, 16, 1, 1),   # 400 row tiles: stream-K, one CTA per SM with a deep ring
-    ("gateup", 128, 128, 1, 1), # many tiles: token tiles of 128
-    ("down", 256, 128, 1, 1),   # a 94 MB weight with 160 tiles of 64: tiles of 128
-    ("q", 256, 64, 1, 1),       # a 30 MB weight: its repeated reads stay in L2, tiles of 64
+@pytest.mark.parametrize("name,M,npad,S,cps,pair", [
+    ("qkv", 16, 16, 2, 2, 0),      # the decode bench launch: clusters of 2, two CTAs per SM
+    ("o", 16, 16, 4, 2, 0),        # o_proj: clusters of 4
+    ("q", 64, 64, 2, 1, 0),
+    ("q", 128, 64, 2, 2, 0),       # 128 tiles of 64 tokens: clusters only with two CTAs per SM
+    ("gateup", 16, 16, 1, 1, 0),   # 400 row tiles: stream-K, one CTA per SM with a deep ring
+    ("gateup", 128, 128, 1, 1, 0), # many tiles: token tiles of 128
+    ("down", 256, 128, 1, 1, 0),   # a 94 MB weight with 160 tiles of 64: tiles of 128
+    ("q", 256, 64, 1, 1, 0),       # a 30 MB weight: its repeated reads stay in L2, tiles of 64
 ])
-def test_plan_choices(name, M, npad, S, cps):
+def test_plan_choices(name, M, npad, S, cps, pair):
     p = spense.plan_shapes(SHAPES[name], M, SMS)
-    assert (p["npad"], p["cluster"], p["ctas_per_sm"]) == (npad, S, cps)
+    assert (p["npad"], p["cluster"], p["ctas_per_sm"], p["pair"]) == (npad, S, cps, pair)
 
 
 def test_plan_workspace_layout():
@@ -112,8 +121,9 @@ def test_plan_workspace_layout():
     for name in ("qkv", "gateup", "down", "split"):
         for M in (1, 16, 256, 600):
             p = spense.plan_shapes(SHAPES[name], M, SMS)
-            counters = -(-p["tiles"] * 4 // 256) * 256
-            partials = 0 if p["cluster"] > 1 else p["grid"] * 2 * p["npad"] * 128 * 4
+            ctas = 2 if p["pair"] else 1  # CTAs per work unit
+            counters = -(-p["tiles"] * ctas * 4 // 256) * 256
+            partials = 0 if p["cluster"] > 1 else p["grid"] * ctas * 2 * p["npad"] * 128 * 4
             assert p["workspace_bytes"] == 256 + counters + partials
             seen.add(p["cluster"] > 1)
     assert seen == {True, False}
