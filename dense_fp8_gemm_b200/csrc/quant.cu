@@ -23,7 +23,7 @@
 namespace spense {
 namespace {
 
-constexpr int kQuantThreads = 256;
+constexpr int kQuantThreads = 512;
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
 
@@ -42,17 +42,38 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   if ((threadIdx.x & 31) == 0) red[w] = v;
   __syncthreads();
   float r = 0.0f;
+#pragma unroll
   for (int i = 0; i < kQuantThreads / 32; ++i) r = fmaxf(r, red[i]);
   return r;
 }
 
+// Sixteen quantised codes of one 16-column output chunk from its 16 source values.
+__device__ __forceinline__ uint4 quantize16(const float (&f)[16], float s) {
+  uint32_t o[4];
+#pragma unroll
+  for (int h = 0; h < 4; ++h) {
+    const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f[4 * h], s), __fdiv_rn(f[4 * h + 1], s));
+    const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f[4 * h + 2], s), __fdiv_rn(f[4 * h + 3], s));
+    o[h] = lo | (hi << 16);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // Each row is split over C CTAs (C = 1 .. 8; more CTAs per row when there are
 // few rows). CTA c writes the 16-column output chunks [K16 c / C, K16 (c + 1) /
-// C) of the row. Every CTA reads the whole row to take its absmax itself (the
-// C - 1 extra reads of a row hit L2; no CTA waits for another), and with a
-// gather it keeps the row in shared memory and gathers from there. Rows too
-// long for shared memory gather from global memory instead (the packed order
-// is two ascending runs, so those loads mostly share cache lines).
+// C) of the row, one chunk per thread per round. Every CTA reads the whole row
+// to take its absmax itself (the C - 1 extra reads of a row hit L2; no CTA
+// waits for another), and with a gather it keeps the row in shared memory and
+// gathers from there. Rows too long for shared memory gather from global
+// memory instead (the packed order is two ascending runs, so those loads
+// mostly share cache lines).
+//
+// At decode sizes the kernel is a chain of memory latencies, so it is cut to
+// as few as possible: the packed order of a thread's first chunk belongs to the
+// weight, not to the previous kernel, so it is fetched before waiting for that
+// kernel; the row is read in one round (eight 16-byte loads in flight per
+// thread, 512 threads: rows up to 32768 columns); then one reduction, and the
+// codes are computed from shared memory or L2.
 // K % 16 == 0; X rows 16-byte aligned; Xq rows 16-byte aligned.
 template <bool kGather, bool kStaged>
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t* __restrict__ X, int64_t K,
@@ -62,11 +83,17 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t*
   extern __shared__ uint4 qsmem[];  // kStaged: the row, K bf16
   __shared__ float red[kQuantThreads / 32];
   pdl_trigger();  // the GEMM that reads Xq may start prefetching its weights
-  pdl_wait();     // X may be written by the previous kernel
   const int64_t m = blockIdx.x / C;
   const int c = static_cast<int>(blockIdx.x % C);
   const int64_t k16 = K / 16;
   const int64_t j0 = k16 * c / C, j1 = k16 * (c + 1) / C;  // this CTA's 16-column chunks
+  int4 cs0[4];  // gather: source columns of this thread's first chunk
+  if (kGather && j0 + threadIdx.x < j1) {
+    const int4* pj = reinterpret_cast<const int4*>(perm + (j0 + threadIdx.x) * 16);
+#pragma unroll
+    for (int h = 0; h < 4; ++h) cs0[h] = __ldg(pj + h);
+  }
+  pdl_wait();  // X may be written by the previous kernel
   const uint16_t* xrow = X + m * K;
   const uint4* xr = reinterpret_cast<const uint4*>(xrow);
   float amax = 0.0f;
@@ -95,61 +122,39 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const uint16_t*
   if (c == 0 && threadIdx.x == 0) s_out[m] = s;
   const uint16_t* src = kStaged ? reinterpret_cast<const uint16_t*>(qsmem) : xrow;
   uint4* qr = reinterpret_cast<uint4*>(Xq + m * K);
-  // Four 16-column chunks per thread per round: all their loads are issued
-  // before any is used, so a round costs one memory latency, not four.
-  constexpr int kU = 4;
-  for (int64_t i0 = j0 + threadIdx.x; i0 < j1; i0 += kU * kQuantThreads) {
-    uint4 raw[kU][2];  // plain: the 16 bf16 of each chunk
-    int4 cs[kU][4];    // gather: the 16 source columns of each chunk
+  for (int64_t i = j0 + threadIdx.x; i < j1; i += kQuantThreads) {
+    float f[16];
+    if (kGather) {
+      int4 cs[4];
+      if (i == j0 + threadIdx.x) {
 #pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t i = i0 + static_cast<int64_t>(u) * kQuantThreads;
-      if (i < j1) {
-        if (kGather) {
-          const int4* pj = reinterpret_cast<const int4*>(perm + i * 16);
-#pragma unroll
-          for (int h = 0; h < 4; ++h) cs[u][h] = __ldg(pj + h);
-        } else {
-          raw[u][0] = __ldg(xr + 2 * i);
-          raw[u][1] = __ldg(xr + 2 * i + 1);
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kU; ++u) {
-      const int64_t i = i0 + static_cast<int64_t>(u) * kQuantThreads;
-      if (i >= j1) break;
-      float f[16];
-      if (kGather) {
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          f[4 * h + 0] = bf16_bits_to_float(kStaged ? src[cs[u][h].x] : __ldg(src + cs[u][h].x));
-          f[4 * h + 1] = bf16_bits_to_float(kStaged ? src[cs[u][h].y] : __ldg(src + cs[u][h].y));
-          f[4 * h + 2] = bf16_bits_to_float(kStaged ? src[cs[u][h].z] : __ldg(src + cs[u][h].z));
-          f[4 * h + 3] = bf16_bits_to_float(kStaged ? src[cs[u][h].w] : __ldg(src + cs[u][h].w));
-        }
+        for (int h = 0; h < 4; ++h) cs[h] = cs0[h];
       } else {
-        const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
-                               raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+        const int4* pj = reinterpret_cast<const int4*>(perm + i * 16);
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          f[2 * h] = bf16_bits_to_float(w[h] & 0xFFFFu);
-          f[2 * h + 1] = bf16_bits_to_float(w[h] >> 16);
-        }
+        for (int h = 0; h < 4; ++h) cs[h] = __ldg(pj + h);
       }
-      uint32_t o[4];
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        const uint32_t lo = cvt_e4m3x2(__fdiv_rn(f[4 * h], s), __fdiv_rn(f[4 * h + 1], s));
-        const uint32_t hi = cvt_e4m3x2(__fdiv_rn(f[4 * h + 2], s), __fdiv_rn(f[4 * h + 3], s));
-        o[h] = lo | (hi << 16);
+        f[4 * h + 0] = bf16_bits_to_float(kStaged ? src[cs[h].x] : __ldg(src + cs[h].x));
+        f[4 * h + 1] = bf16_bits_to_float(kStaged ? src[cs[h].y] : __ldg(src + cs[h].y));
+        f[4 * h + 2] = bf16_bits_to_float(kStaged ? src[cs[h].z] : __ldg(src + cs[h].z));
+        f[4 * h + 3] = bf16_bits_to_float(kStaged ? src[cs[h].w] : __ldg(src + cs[h].w));
       }
-      qr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+      const uint4 r0 = __ldg(xr + 2 * i), r1 = __ldg(xr + 2 * i + 1);
+      const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        f[2 * h] = bf16_bits_to_float(w[h] & 0xFFFFu);
+        f[2 * h + 1] = bf16_bits_to_float(w[h] >> 16);
+      }
     }
+    qr[i] = quantize16(f, s);
   }
 }
 
-// Shared memory for a staged row: at most 56 KB, so four CTAs fit per SM.
+// Shared memory for a staged row: at most 56 KB, so four CTAs (of 512 threads) fit per SM.
 constexpr int64_t kQuantStageBytes = 56 * 1024;
 
 }  // namespace
@@ -159,9 +164,12 @@ cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32
   if (M == 0) return cudaSuccess;
   // CTAs per row: one once the rows alone cover the SMs (every extra CTA of a
   // row reads the row again); otherwise enough for two CTAs per SM, at most 8
-  // and at most one per 16-column chunk.
+  // and at most one per 16-column chunk. Measured at 25600 columns, back to
+  // back: 1, 2, 4, 8, 16 CTAs per row take 7.8, 6.3, 4.7, 3.8, 3.5 us at 16
+  // tokens and 8.5, 6.8, 4.8, 4.0, 6.6 us at 32 tokens.
   int64_t C = M >= sms ? 1 : (2 * static_cast<int64_t>(sms) + M - 1) / M;
   C = C < 1 ? 1 : (C > 8 ? 8 : C);
+
   while (C > 1 && K / 16 < C) --C;
   const unsigned int grid = static_cast<unsigned int>(M * C);
   const int ci = static_cast<int>(C);
