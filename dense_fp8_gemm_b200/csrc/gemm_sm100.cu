@@ -630,65 +630,75 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       stage_sx(m0);
       const GemmMember& mb = p.mem[member_of(p, n_tile)];
       const int m_valid = min(p.npad, p.M - m0);
-      const int n = (P * (n_tile - mb.tile_begin) + static_cast<int>(prank)) * kTileRows + row;
-      const bool row_ok = n < mb.N;
-      const float sw = row_ok ? __ldg(mb.s_w + n) : 0.0f;
       int nb_t;
       const int tb = tile_block0(p, t, &nb_t);
       const int g_lo = block_owner(p, tb);
       const int g_hi = block_owner(p, tb + nb_t - 1);
       const int lo_slot = (p.cta_start[g_lo] >= tb) ? 0 : 1;
-      // The contributors' partials of this CTA's rows: work unit gg's CTA of
-      // the same rank in the pair (CTA gg x P + rank).
-      const float* lo_part = p.partials + (static_cast<size_t>(g_lo * P + prank) * 2 + lo_slot) * slot_elems +
-                             static_cast<size_t>(row) * p.npad;
-      const float* next_part = p.partials + (static_cast<size_t>((g_lo + 1) * P + prank) * 2) * slot_elems +
-                               static_cast<size_t>(row) * p.npad;
+      // Partial slots are token-major, [npad tokens][128 rows]. For the sum the
+      // 128 threads are remapped: lane l takes rows 4l .. 4l + 3 and warp w
+      // tokens 4w .. 4w + 3 of every 16-token chunk, so each access is a
+      // 16-byte load (a warp covers one token's 128 rows) and each output a
+      // 4-row 8-byte store.
+      const int r0 = (et & 31) * 4;
+      const int tq = (et >> 5) * 4;
+      const int n0 = (P * (n_tile - mb.tile_begin) + static_cast<int>(prank)) * kTileRows + r0;
+      float sw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sw[i] = n0 + i < mb.N ? __ldg(mb.s_w + n0 + i) : 0.0f;
+      const bool vec = n0 + 4 <= mb.N && (mb.ldy % 4) == 0;
+      const float* lo_part = p.partials + (static_cast<size_t>(g_lo * P + prank) * 2 + lo_slot) * slot_elems + r0;
+      const float* next_part = p.partials + (static_cast<size_t>((g_lo + 1) * P + prank) * 2) * slot_elems + r0;
       const size_t stride = static_cast<size_t>(2 * P) * slot_elems;  // from contributor gg to gg + 1 (slot 0)
       const int others = g_hi - g_lo;
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
-        const int nq = min(4, (m_valid - c0 + 3) >> 2);  // float4 groups holding valid tokens
         float4 a[4], b[4], c[4];
+        const int mb0 = c0 + tq;  // this warp's first token of the chunk
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (q < nq) a[q] = __ldcg(reinterpret_cast<const float4*>(lo_part + c0) + q);
+        for (int j = 0; j < 4; ++j)
+          if (mb0 + j < m_valid)
+            a[j] = __ldcg(reinterpret_cast<const float4*>(lo_part + static_cast<size_t>(mb0 + j) * kTileRows));
         int k = 0;
         for (; k + 2 <= others; k += 2) {
-          const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
-          const float4* pc = reinterpret_cast<const float4*>(next_part + (k + 1) * stride + c0);
+          const float* pb = next_part + k * stride;
+          const float* pc = pb + stride;
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (q < nq) {
-              b[q] = __ldcg(pb + q);
-              c[q] = __ldcg(pc + q);
+          for (int j = 0; j < 4; ++j)
+            if (mb0 + j < m_valid) {
+              b[j] = __ldcg(reinterpret_cast<const float4*>(pb + static_cast<size_t>(mb0 + j) * kTileRows));
+              c[j] = __ldcg(reinterpret_cast<const float4*>(pc + static_cast<size_t>(mb0 + j) * kTileRows));
             }
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (q < nq) {
-              a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
-              a[q].x += c[q].x; a[q].y += c[q].y; a[q].z += c[q].z; a[q].w += c[q].w;
+          for (int j = 0; j < 4; ++j)
+            if (mb0 + j < m_valid) {
+              a[j].x += b[j].x; a[j].y += b[j].y; a[j].z += b[j].z; a[j].w += b[j].w;
+              a[j].x += c[j].x; a[j].y += c[j].y; a[j].z += c[j].z; a[j].w += c[j].w;
             }
         }
         if (k < others) {
-          const float4* pb = reinterpret_cast<const float4*>(next_part + k * stride + c0);
+          const float* pb = next_part + k * stride;
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (q < nq) {
-              b[q] = __ldcg(pb + q);
-              a[q].x += b[q].x; a[q].y += b[q].y; a[q].z += b[q].z; a[q].w += b[q].w;
+          for (int j = 0; j < 4; ++j)
+            if (mb0 + j < m_valid) {
+              b[j] = __ldcg(reinterpret_cast<const float4*>(pb + static_cast<size_t>(mb0 + j) * kTileRows));
+              a[j].x += b[j].x; a[j].y += b[j].y; a[j].z += b[j].z; a[j].w += b[j].w;
             }
         }
-        if (row_ok) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float r4[4] = {a[q].x, a[q].y, a[q].z, a[q].w};
+        for (int j = 0; j < 4; ++j) {
+          const int m = mb0 + j;
+          if (m >= m_valid) continue;
+          const float sx = m0 == staged_m0 ? bars->sx[m] : __ldg(p.s_x + m0 + m);
+          const uint32_t v0 = to_bf16_bits(a[j].x * sw[0] * sx), v1 = to_bf16_bits(a[j].y * sw[1] * sx);
+          const uint32_t v2 = to_bf16_bits(a[j].z * sw[2] * sx), v3 = to_bf16_bits(a[j].w * sw[3] * sx);
+          uint16_t* yrow = mb.y + static_cast<size_t>(m0 + m) * mb.ldy;
+          if (vec) {
+            *reinterpret_cast<uint2*>(yrow + n0) = make_uint2(v0 | (v1 << 16), v2 | (v3 << 16));
+          } else {
+            const uint32_t vv[4] = {v0, v1, v2, v3};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int m = c0 + 4 * q + i;
-              if (q < nq && m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] =
-                    to_bf16_bits(r4[i] * sw * (m0 == staged_m0 ? bars->sx[m] : __ldg(p.s_x + m0 + m)));
-            }
+            for (int i = 0; i < 4; ++i)
+              if (n0 + i < mb.N) yrow[n0 + i] = static_cast<uint16_t>(vv[i]);
           }
         }
       }
@@ -836,13 +846,12 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       if (!ptx::named_bar_and(1, 128, got)) break;
       ptx::tc_fence_after();
       const uint32_t taddr = lane_base + acc * static_cast<uint32_t>(p.npad);
-      // Partials are stored [CTA][slot][row][npad]: slot 0 for the tile holding the
-      // CTA's first block, slot 1 for the tile holding its last block.
+      // Partials are stored [CTA][slot][npad][row] (token-major): slot 0 for the
+      // tile holding the CTA's first block, slot 1 for the tile holding its last block.
       float* part = nullptr;
       if (!whole) {
         const int slot = (b0 >= tb) ? 0 : 1;
-        part = p.partials + (static_cast<size_t>(g * P + prank) * 2 + slot) * slot_elems +
-               static_cast<size_t>(row) * p.npad;
+        part = p.partials + (static_cast<size_t>(g * P + prank) * 2 + slot) * slot_elems + row;  // token-major
       }
       for (int c0 = 0; c0 < m_valid; c0 += 16) {
         uint32_t v[16];
@@ -858,12 +867,10 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             }
           }
         } else {
-          float4* dst = reinterpret_cast<float4*>(part + c0);
+          // token-major partial: consecutive threads (rows) store consecutive words
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (c0 + 4 * q < m_valid)
-              __stcg(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                                          __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+          for (int i = 0; i < 16; ++i)
+            if (c0 + i < m_valid) __stcg(part + static_cast<size_t>(c0 + i) * kTileRows, __uint_as_float(v[i]));
         }
       }
       ptx::tc_fence_before();
