@@ -43,9 +43,24 @@ def test_summary_command_is_reproducible(path):
             assert f'"{opt}"' in source, f"{opt} is not an option of {os.path.basename(target)}"
 
 
-def test_traffic_record_names_its_sources():
-    rec = json.load(open(os.path.join(ROOT, "profiles", "spense_gemm_attn32b_m16_traffic.txt")))
+TRAFFIC = sorted(glob.glob(os.path.join(ROOT, "profiles", "*_traffic.txt")))
+
+
+@pytest.mark.parametrize("path", TRAFFIC, ids=os.path.basename)
+def test_traffic_record_names_its_sources(path):
+    rec = json.load(open(path))
     assert re.fullmatch(r"[0-9a-f]{64}", rec["kernel_source_sha256"])
     for name in rec["kernel_sources"]:
         assert os.path.isfile(os.path.join(ROOT, "dense_fp8_gemm_b200", "csrc", name)), name
-    assert rec["dram_bytes_per_launch_avg"] > 0
+    per = rec["dram_bytes_per_launch"]
+    assert rec["dram_bytes_per_launch_avg"] == sum(per.values()) // len(per) > 0
+    assert "--clock-control none" in rec["source"]
+
+
+def test_bench_workloads_have_a_traffic_record():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    names = {os.path.basename(p) for p in TRAFFIC}
+    for wl in bench.STACKS:
+        assert f"spense_gemm_{wl}_m16_traffic.txt" in names
