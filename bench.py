@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--dense-frac", type=float, default=0.25)
     ap.add_argument("--cpu-seconds", type=float, default=20.0, help="CPU-baseline budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cublas", action="store_true",
+                    help="skip the reference line of cuBLASLt dense FP8 (torch._scaled_mm) on the same step")
     ap.add_argument("--op", choices=["gemm", "quantize", "score", "glu"], default="gemm",
                     help="gemm: the hybrid GEMM over a decoder stack (default, the headline); quantize: the "
                          "per-token FP8 quantisation with the SpenseGPT+ column order fused in; score: the "
@@ -409,18 +411,28 @@ def run_spense(args):
 
     # ---- weights: every layer distinct, drawn on the GPU, packed twice: the
     # Spense format (dense_frac of the columns dense, the rest 2:4) and all
-    # dense (the same kernel on the dense FP8 matrix, Kd = K).
+    # dense (the same kernel on the dense FP8 matrix, Kd = K). For the
+    # cuBLASLt reference line the same dense FP8 matrices are also kept as
+    # plain tensors, the weights of a launch group concatenated along N.
+    use_cublas = not args.no_cublas and hasattr(torch, "_scaled_mm")
     t_gen = time.perf_counter()
     arms = {"spense": [], "dense": []}
+    cublas_w = []  # per layer, per launch group: (W e4m3 [N_g, K], s_w [1, N_g])
     for L in range(layers):
-        sp, dn = [], []
+        sp, dn, raw = [], [], []
         for i, (_, N, K) in enumerate(wl.shapes):
             q, sc = synth.device_fp8_rows(wl.seed, workloads.weight_id(i, L), (N, K), wl.w_std, dev)
             sp.append(spense.pack(q, sc, Kd=workloads.dense_count(K, args.dense_frac)))
             dn.append(spense.pack(q, sc, Kd=K))
+            if use_cublas:
+                raw.append((q, sc))
             del q, sc
         arms["spense"].append(sp)
         arms["dense"].append(dn)
+        if use_cublas:
+            cublas_w.append([(torch.cat([raw[i][0] for i in g]).view(torch.float8_e4m3fn),
+                              torch.cat([raw[i][1] for i in g]).view(1, -1)) for g in groups])
+            del raw
     torch.cuda.synchronize()
     gen_s = time.perf_counter() - t_gen
 
@@ -512,6 +524,38 @@ def run_spense(args):
         per_group[name] = {"us_per_launch": us * 1e6, "GBps": byt / us / 1e9, "frac": byt / us / 1e9 / peak,
                            "dense_fp8_us": res["dense"][0] * 1e6, "speedup_vs_dense_fp8": res["dense"][0] / us}
 
+    # ---- reference line: cuBLASLt dense FP8 (torch._scaled_mm, rowwise fp32
+    # scales, bf16 out) on the same step's dense FP8 matrices, one call per
+    # launch group, in one CUDA graph like the Spense step. A library GEMM,
+    # timed for context only.
+    cublas = None
+    if use_cublas:
+        try:
+            xs8 = [X[gi][:M0].view(torch.float8_e4m3fn) for gi in range(len(groups))]
+            sxs = [SX[gi][:M0].view(-1, 1) for gi in range(len(groups))]
+
+            def cublas_step():
+                for Lw in cublas_w:
+                    for gi, (w8, sw) in enumerate(Lw):
+                        torch._scaled_mm(xs8[gi], w8.t(), scale_a=sxs[gi], scale_b=sw, out_dtype=torch.bfloat16)
+
+            cublas_step()
+            torch.cuda.synchronize()
+            g_cb = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_cb, stream=stream):
+                cublas_step()
+            g_cb.replay()
+            torch.cuda.synchronize()
+            t_cb = timed(g_cb, sub_steps, 2) / sub_steps
+            del g_cb
+            cublas = {"ms_per_step": t_cb * 1e3, "GBps": step_bytes(args, dense=True) / t_cb / 1e9,
+                      "spense_speedup": t_cb / (t_sp / args.steps),
+                      "call": "torch._scaled_mm(X e4m3 [M,K], W e4m3 [N,K]^T, rowwise fp32 scales) -> bf16, "
+                              "one call per launch group, 64 layers in one CUDA graph"}
+        except Exception as e:  # the reference line is context only: report why it is missing
+            cublas = {"unavailable": f"{type(e).__name__}: {str(e)[:200]}"}
+        del cublas_w
+
     # ---- other token counts on the same weights
     per_m = {}
     for M in Ms[1:]:
@@ -585,6 +629,7 @@ def run_spense(args):
                          "kernel": "spense_gemm_kernel", "avg_launch_us": avg_launch_s * 1e6,
                          "bytes_per_launch": bytes_per_launch, "launches_per_step": launches_per_step},
             "per_launch_group": per_group,
+            "cublas_dense_fp8": cublas,
             "per_tokens": per_m,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
