@@ -342,7 +342,15 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
       if (!(mode > 1 || fills || small)) continue;
       int st, na;
       uint32_t co;
-      if (fit_ring(cps, static_cast<uint32_t>(S - 1) * kTileRows * pl.npad * 4u, &st, &na, &co)) return S;
+      if (!fit_ring(cps, static_cast<uint32_t>(S - 1) * kTileRows * pl.npad * 4u, &st, &na, &co)) continue;
+      // A two-stage ring only pays when each CTA streams few blocks: q_proj
+      // 8192x5120 at 128 tokens (about 13 blocks per CTA) 42.5 -> 16.1 us
+      // with it, but down 5120x27648 at 128 tokens (about 67 per CTA) took
+      // 53.8 us against 40.7 us as stream-K with a deep ring.
+      int max_blocks = 0;
+      for (int i = 0; i < count; ++i) max_blocks = std::max(max_blocks, pl.mem_nsb[i] + pl.mem_ndb[i]);
+      if (st < 3 && max_blocks > 16 * S) continue;
+      return S;
     }
     return 1;
   };

@@ -107,6 +107,8 @@ def test_plan_invariants(name, M):
     ("gateup", 128, 128, 1, 1, 0), # many tiles: token tiles of 128
     ("down", 256, 128, 1, 1, 0),   # a 94 MB weight with 160 tiles of 64: tiles of 128
     ("q", 256, 64, 1, 1, 0),       # a 30 MB weight: its repeated reads stay in L2, tiles of 64
+    ("down36", 128, 64, 1, 1, 0),  # 135 blocks per tile: no two-stage cluster ring, stream-K with a deep one
+    ("o36", 16, 16, 4, 2, 0),      # three stages at two CTAs per SM: clusters of 4 stay
 ])
 def test_plan_choices(name, M, npad, S, cps, pair):
     p = spense.plan_shapes(SHAPES[name], M, SMS)
