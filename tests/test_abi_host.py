@@ -205,3 +205,20 @@ def test_glu_order_rejects_bad_sets(L):
         with pytest.raises(spense.SpenseError) as e:
             spense.glu_order(I, d)
         assert e.value.code == code, (I, d, e.value)
+
+
+def test_grouped_host_rejects_bad_arguments(L):
+    """spense_gemm_grouped_host checks its flags and pointers before any device
+    work: unknown flags, NULL input or output, and (for device-side buffers)
+    misalignment come back as status codes."""
+    v = lambda a: ctypes.c_void_p(a) if a else None
+    h = (ctypes.c_void_p * 1)(0x10)
+    y = (ctypes.c_void_p * 1)(0x3000)
+    def call(X=0x1000, sx=0x2000, Ys=y, ws=0x4000, flags=0):
+        return L.spense_gemm_grouped_host(h, 1, v(X), v(sx), 4, Ys, v(ws), 1 << 20, flags, None)
+    assert call(flags=0x8) == 1 and b"flags" in L.spense_last_error()
+    assert call(X=0) == 1 and call(sx=0) == 1 and call(Ys=None) == 1
+    assert call(X=0x1004) == 3                       # a device X must be 16-byte aligned
+    assert call(sx=0x2002) == 3
+    assert call(ws=0) == 7                           # no workspace
+    assert L.spense_gemm_grouped_host_workspace_size(None, 1, 4) == 0

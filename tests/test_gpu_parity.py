@@ -161,6 +161,41 @@ def test_gemm_is_deterministic_and_host_path_agrees():
     assert torch.equal(Yh.view(torch.int16), Y1.cpu().view(torch.int16))
 
 
+@pytest.mark.parametrize("flags", ["x", "y", "xy", "none"])
+def test_grouped_host_entry_point_equals_the_device_path(flags):
+    """spense_gemm_grouped_host with the input in host memory (GEMM_HOST_X), the
+    outputs in host memory (GEMM_HOST_Y), both, or neither: the same launch as
+    spense_gemm_grouped on device buffers, so the outputs are equal bit for bit;
+    the copies run inside the call (a decode step issued from host buffers)."""
+    M, K, Kd = 16, 1024, 256
+    Ns = (384, 128, 128)
+    X, s_x = synth.quantize_rows(synth.normal(61, 1, (M, K), 1.0))
+    pws = []
+    for i, N in enumerate(Ns):
+        W, s_w = synth.quantize_rows(synth.normal(61, 10 + i, (N, K), 0.02))
+        pws.append(spense.pack(_dev(W), _dev(s_w), Kd=Kd))
+    Xd, sxd = _dev(X), _dev(s_x)
+    ref = spense.gemm_grouped(pws, Xd, sxd)
+    f = (spense.GEMM_HOST_X if "x" in flags else 0) | (spense.GEMM_HOST_Y if "y" in flags else 0)
+    ws = spense.new_workspace(spense.grouped_host_workspace_size(pws, M))
+    xin = torch.from_numpy(X).pin_memory() if "x" in flags else Xd
+    sin = torch.from_numpy(s_x).pin_memory() if "x" in flags else sxd
+    if "y" in flags:
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for N in Ns]
+    else:
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device="cuda") for N in Ns]
+    for _ in range(2):  # twice: the second call reuses the cached launch and the staging areas
+        for Y in Ys:
+            Y.fill_(float("nan"))
+        spense.gemm_grouped_host(pws, xin, sin, Ys, ws, f)
+        torch.cuda.synchronize()
+        for Y, R in zip(Ys, ref):
+            assert torch.equal(Y.cpu().view(torch.int16), R.cpu().view(torch.int16)), flags
+    assert spense.workspace_status(ws) == 0
+    for pw in pws:
+        pw.free()
+
+
 def test_spenseplus_with_tail_list_equals_spensegpt():
     M, N, K, Kd = 8, 256, 1024, 256
     X, s_x, W, s_w, _ = _make(41, M, N, K, Kd)
