@@ -257,10 +257,19 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // weight rows, and token tiles of up to 256 tokens read each weight once.
   const int pk = pair_knob();
   pl.pair = (x_warp() && (pk == 2 || (pk == 1 && M > 64))) ? 1 : 0;
-  const int T = token_tile_knob() != 0
-                    ? token_tile_knob()
-                    : (pl.pair ? kMaxTokenTile
-                               : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128));
+  int T = token_tile_knob() != 0
+              ? token_tile_knob()
+              : (pl.pair ? kMaxTokenTile
+                         : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128));
+  // Tiles of 128 tokens that leave most CTAs straddling two tiles (fewer than
+  // 1.5 tiles per SM) while tiles of 96 would give each about two: take 96
+  // (q/k/v 12288x5120 at 256 tokens 35.3 -> 28.4 us; weights that stay at
+  // fewer than 1.5 tiles per SM either way were slower with 96). Only for a
+  // weight of at most 64 MB, whose re-reads by the extra token tile stay in L2.
+  if (token_tile_knob() == 0 && !pl.pair && T == 128 && M > 128 && weight_units * 4096ll <= (64ll << 20)) {
+    const long long t128 = row_tiles * ((M + 127) / 128), t96 = row_tiles * ((M + 95) / 96);
+    if (2 * t128 < 3LL * sms && 2 * t96 >= 3LL * sms) T = 96;
+  }
   pl.npad = M > T ? T : static_cast<int>(round_up(static_cast<size_t>(M), 16));
   // rows one activation box loads: the valid rows of the token tile, or in
   // pair mode this CTA's half of it (rows past M read as zeros)

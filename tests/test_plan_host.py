@@ -28,6 +28,7 @@ SHAPES = {
     "o36": [(5120, 10240, 2560)],
     "gateup36": [(55296, 5120, 1280)],
     "down36": [(5120, 27648, 6912)],
+    "qkv36": [(10240, 5120, 1280), (1024, 5120, 1280), (1024, 5120, 1280)],
     "split": [(19200, 5120, 0), (6400, 5120, 5120)],           # output-split: 2:4 rows, dense rows
     "ragged": [(1000, 1024, 256), (136, 1024, 256)],
 }
@@ -109,6 +110,8 @@ def test_plan_invariants(name, M):
     ("q", 256, 64, 1, 1, 0),       # a 30 MB weight: its repeated reads stay in L2, tiles of 64
     ("down36", 128, 64, 1, 1, 0),  # 135 blocks per tile: no two-stage cluster ring, stream-K with a deep one
     ("o36", 16, 16, 4, 2, 0),      # three stages at two CTAs per SM: clusters of 4 stay
+    ("qkv36", 256, 96, 1, 1, 0),   # 128-token tiles: 1.3 per SM; 96: about 2 (45 MB stays in L2)
+    ("down36", 600, 128, 1, 1, 0), # 102 MB: its re-reads would leave L2, tiles of 128 stay
 ])
 def test_plan_choices(name, M, npad, S, cps, pair):
     p = spense.plan_shapes(SHAPES[name], M, SMS)
