@@ -340,6 +340,8 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // area (S - 1 partials of 128 rows x npad floats) comes out of the ring.
   // Returns the largest such S for `cps` CTAs per SM, or 1.
   const int mode = cluster_mode();
+  int max_blocks = 0;  // blocks per tile of the member with the longest K
+  for (int i = 0; i < count; ++i) max_blocks = std::max(max_blocks, pl.mem_nsb[i] + pl.mem_ndb[i]);
   auto cluster_for = [&](int cps) {
     const long long slots = slots_for(cps);
     if (mode == 0 || pl.tiles * 2 > slots || pl.npad > 64) return 1;
@@ -356,9 +358,13 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
       // 8192x5120 at 128 tokens (about 13 blocks per CTA) 42.5 -> 16.1 us
       // with it, but down 5120x27648 at 128 tokens (about 67 per CTA) took
       // 53.8 us against 40.7 us as stream-K with a deep ring.
-      int max_blocks = 0;
-      for (int i = 0; i < count; ++i) max_blocks = std::max(max_blocks, pl.mem_nsb[i] + pl.mem_ndb[i]);
       if (st < 3 && max_blocks > 16 * S) continue;
+      // Clusters that leave over 40 % of the SMs idle lose to stream-K over
+      // all of them when each clustered CTA would stream a long K range:
+      // down 5120x27648 (135 blocks per tile, clusters of 2 on 80 SMs) at 32
+      // and 64 tokens 30.8 -> 24.5 us and 32.6 -> 27.3 us as stream-K; o_proj
+      // 5120x10240 (50 blocks per tile) stays faster in clusters.
+      if (10LL * pl.tiles * S < 6LL * sms && max_blocks > 32 * S) continue;
       return S;
     }
     return 1;
@@ -380,6 +386,10 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
       cps = 3 - cps;
       pl.cluster = cluster_for(cps);
     }
+    // Few long tiles left to stream-K: one CTA per SM with a deeper ring and
+    // half the partials (down 5120x27648 at 32 tokens 24.5 us against 25.1 us
+    // at two per SM).
+    if (pl.cluster == 1 && knob == 0 && 10LL * pl.tiles < 6LL * sms && max_blocks > 64) cps = 1;
   }
   pl.recv_bytes = pl.cluster > 1 ? static_cast<uint32_t>(pl.cluster - 1) * kTileRows * pl.npad * 4u : 0u;
   if (!fit_ring(cps, pl.recv_bytes, &pl.stages, &pl.nacc, &pl.tmem_cols)) {

@@ -112,6 +112,9 @@ def test_plan_invariants(name, M):
     ("o36", 16, 16, 4, 2, 0),      # three stages at two CTAs per SM: clusters of 4 stay
     ("qkv36", 256, 96, 1, 1, 0),   # 128-token tiles: 1.3 per SM; 96: about 2 (45 MB stays in L2)
     ("down36", 600, 128, 1, 1, 0), # 102 MB: its re-reads would leave L2, tiles of 128 stay
+    ("down36", 32, 32, 1, 1, 0),   # 40 tiles of 135 blocks: stream-K over every SM, not clusters of 2 on 80
+    ("down36", 64, 64, 1, 1, 0),
+    ("o36", 64, 64, 2, 1, 0),      # 50 blocks per tile: clusters of 2 stay
 ])
 def test_plan_choices(name, M, npad, S, cps, pair):
     p = spense.plan_shapes(SHAPES[name], M, SMS)
