@@ -56,7 +56,7 @@ namespace {
 
 constexpr uint64_t kWaitLimitNs = 1500000000ull;
 
-struct alignas(8) Barriers {
+struct alignas(16) Barriers {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   uint64_t acc_full[2];
@@ -67,7 +67,9 @@ struct alignas(8) Barriers {
   uint32_t tmem_base;
   int abort_flag;
   int fix_flag;
-  float sx[kMaxTokenTile];  // per-token scales of the token tile being finished
+  int npend;    // stream-K: fix-ups left for the end of the kernel (0 to 2)
+  int pend[2];  // ... their tiles
+  alignas(16) float sx[kMaxTokenTile];  // per-token scales of the token tile being finished
 };
 static_assert(sizeof(Barriers) <= kBarrierBytes, "barrier area too small");
 
@@ -218,6 +220,117 @@ struct BlockWalker {
   }
 };
 
+__device__ __forceinline__ uint16_t to_bf16_bits(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+// The token scales sx[0 .. 15] (staged in shared memory, 16-byte aligned) into
+// registers ahead of a chunk's stores. Read one at a time between the stores,
+// every load waited for the store before it (the compiler cannot tell the
+// staged scales from the outputs apart): a 128-token epilogue took about 4x as
+// long that way.
+__device__ __forceinline__ void load_sx16(const float* sx, float (&s)[16]) {
+  const float4* s4 = reinterpret_cast<const float4*>(sx);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 f = s4[q];
+    s[4 * q] = f.x;
+    s[4 * q + 1] = f.y;
+    s[4 * q + 2] = f.z;
+    s[4 * q + 3] = f.w;
+  }
+}
+
+// Sums the contributors' partials of stream-K tile t in CTA order, applies
+// the scales and stores Y (for a CTA pair: rank prank's 128 rows). Every
+// contributor after g_lo starts inside tile t, so its partial is in slot 0;
+// g_lo uses slot 1 when its range started in an earlier tile. Threads
+// [0, nthr) of the CTA take part (nthr a multiple of 32, tid the caller's
+// index among them). Partial slots are token-major, [npad tokens][128 rows]:
+// lane l sums rows 4l .. 4l + 3 and warp w tokens 4w .. 4w + 3 of every chunk
+// of 4 nthr / 32 tokens, so each access is a 16-byte load (a warp covers one
+// token's 128 rows) and each output a 4-row 8-byte store. sx: the token tile's
+// scales, staged in shared memory.
+__device__ __forceinline__ void fixup_tile(const GemmParams& p, int t, int P, uint32_t prank, int tid, int nthr,
+                                           const float* sx) {
+  const int n_tile = t / p.m_tiles;
+  const int m0 = (t - n_tile * p.m_tiles) * p.npad;
+  const GemmMember& mb = p.mem[member_of(p, n_tile)];
+  const int m_valid = min(p.npad, p.M - m0);
+  int nb_t;
+  const int tb = tile_block0(p, t, &nb_t);
+  const int g_lo = block_owner(p, tb);
+  const int g_hi = block_owner(p, tb + nb_t - 1);
+  const int lo_slot = (p.cta_start[g_lo] >= tb) ? 0 : 1;
+  const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
+  const int r0 = (tid & 31) * 4;
+  const int tq = (tid >> 5) * 4;
+  const int step = 4 * (nthr >> 5);
+  const int n0 = (P * (n_tile - mb.tile_begin) + static_cast<int>(prank)) * kTileRows + r0;
+  float sw[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sw[i] = n0 + i < mb.N ? __ldg(mb.s_w + n0 + i) : 0.0f;
+  const bool vec = n0 + 4 <= mb.N && (mb.ldy % 4) == 0;
+  const float* lo_part = p.partials + (static_cast<size_t>(g_lo * P + prank) * 2 + lo_slot) * slot_elems + r0;
+  const float* next_part = p.partials + (static_cast<size_t>((g_lo + 1) * P + prank) * 2) * slot_elems + r0;
+  const size_t stride = static_cast<size_t>(2 * P) * slot_elems;  // from contributor gg to gg + 1 (slot 0)
+  const int others = g_hi - g_lo;
+  for (int c0 = 0; c0 < m_valid; c0 += step) {
+    float4 a[4], b[4], c[4];
+    const int mb0 = c0 + tq;  // this warp's first token of the chunk
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (mb0 + j < m_valid)
+        a[j] = __ldcg(reinterpret_cast<const float4*>(lo_part + static_cast<size_t>(mb0 + j) * kTileRows));
+    int k = 0;
+    for (; k + 2 <= others; k += 2) {
+      const float* pb = next_part + k * stride;
+      const float* pc = pb + stride;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (mb0 + j < m_valid) {
+          b[j] = __ldcg(reinterpret_cast<const float4*>(pb + static_cast<size_t>(mb0 + j) * kTileRows));
+          c[j] = __ldcg(reinterpret_cast<const float4*>(pc + static_cast<size_t>(mb0 + j) * kTileRows));
+        }
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (mb0 + j < m_valid) {
+          a[j].x += b[j].x; a[j].y += b[j].y; a[j].z += b[j].z; a[j].w += b[j].w;
+          a[j].x += c[j].x; a[j].y += c[j].y; a[j].z += c[j].z; a[j].w += c[j].w;
+        }
+    }
+    if (k < others) {
+      const float* pb = next_part + k * stride;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (mb0 + j < m_valid) {
+          b[j] = __ldcg(reinterpret_cast<const float4*>(pb + static_cast<size_t>(mb0 + j) * kTileRows));
+          a[j].x += b[j].x; a[j].y += b[j].y; a[j].z += b[j].z; a[j].w += b[j].w;
+        }
+    }
+    const float4 s4 = *reinterpret_cast<const float4*>(sx + mb0);  // ahead of the stores (see load_sx16)
+    const float s_tok[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int m = mb0 + j;
+      if (m >= m_valid) continue;
+      const float s = s_tok[j];
+      const uint32_t v0 = to_bf16_bits(a[j].x * sw[0] * s), v1 = to_bf16_bits(a[j].y * sw[1] * s);
+      const uint32_t v2 = to_bf16_bits(a[j].z * sw[2] * s), v3 = to_bf16_bits(a[j].w * sw[3] * s);
+      uint16_t* yrow = mb.y + static_cast<size_t>(m0 + m) * mb.ldy;
+      if (vec) {
+        *reinterpret_cast<uint2*>(yrow + n0) = make_uint2(v0 | (v1 << 16), v2 | (v3 << 16));
+      } else {
+        const uint32_t vv[4] = {v0, v1, v2, v3};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (n0 + i < mb.N) yrow[n0 + i] = static_cast<uint16_t>(vv[i]);
+      }
+    }
+  }
+  if (tid == 0) p.counters[t * P + prank] = 0u;  // re-arm for the next launch (ordered by the kernel boundary)
+}
+
 // Ring position: stage index and the parity of its current use.
 struct Ring {
   uint32_t s = 0, ph = 0, n;
@@ -229,10 +342,6 @@ struct Ring {
     }
   }
 };
-
-__device__ __forceinline__ uint16_t to_bf16_bits(float v) {
-  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
-}
 
 // kPair: the pair-mode instantiation. A kernel holding tcgen05 cta_group::2
 // instructions can only be launched as clusters of CTA pairs, so the
@@ -305,6 +414,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     }
     bars->abort_flag = 0;
     bars->fix_flag = 0;
+    bars->npend = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
@@ -610,6 +720,9 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     const size_t slot_elems = static_cast<size_t>(kTileRows) * p.npad;
+    // This warp's 1 KB of output staging (plans with room for it), after the barrier area.
+    uint16_t* const wstage =
+        p.ystage ? reinterpret_cast<uint16_t*>(smem + recv_off + p.recv_bytes + kBarrierBytes) + quarter * 512 : nullptr;
     // Token scales of the current token tile, staged in shared memory before
     // the accumulator is ready so no global load sits on the epilogue's path.
     int staged_m0 = -1;
@@ -621,88 +734,10 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       staged_m0 = m0;
     };
 
-    // Sum the contributors' partials of tile t in CTA order and store Y. Every
-    // contributor after g_lo starts inside tile t, so its partial is in slot
-    // 0; g_lo uses slot 1 when its range started in an earlier tile.
+    // Fix-up of a shared tile by the epilogue warps while this CTA's MMAs go on.
     auto finish_tile = [&](int t) {
-      const int n_tile = t / p.m_tiles;
-      const int m0 = (t - n_tile * p.m_tiles) * p.npad;
-      stage_sx(m0);
-      const GemmMember& mb = p.mem[member_of(p, n_tile)];
-      const int m_valid = min(p.npad, p.M - m0);
-      int nb_t;
-      const int tb = tile_block0(p, t, &nb_t);
-      const int g_lo = block_owner(p, tb);
-      const int g_hi = block_owner(p, tb + nb_t - 1);
-      const int lo_slot = (p.cta_start[g_lo] >= tb) ? 0 : 1;
-      // Partial slots are token-major, [npad tokens][128 rows]. For the sum the
-      // 128 threads are remapped: lane l takes rows 4l .. 4l + 3 and warp w
-      // tokens 4w .. 4w + 3 of every 16-token chunk, so each access is a
-      // 16-byte load (a warp covers one token's 128 rows) and each output a
-      // 4-row 8-byte store.
-      const int r0 = (et & 31) * 4;
-      const int tq = (et >> 5) * 4;
-      const int n0 = (P * (n_tile - mb.tile_begin) + static_cast<int>(prank)) * kTileRows + r0;
-      float sw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) sw[i] = n0 + i < mb.N ? __ldg(mb.s_w + n0 + i) : 0.0f;
-      const bool vec = n0 + 4 <= mb.N && (mb.ldy % 4) == 0;
-      const float* lo_part = p.partials + (static_cast<size_t>(g_lo * P + prank) * 2 + lo_slot) * slot_elems + r0;
-      const float* next_part = p.partials + (static_cast<size_t>((g_lo + 1) * P + prank) * 2) * slot_elems + r0;
-      const size_t stride = static_cast<size_t>(2 * P) * slot_elems;  // from contributor gg to gg + 1 (slot 0)
-      const int others = g_hi - g_lo;
-      for (int c0 = 0; c0 < m_valid; c0 += 16) {
-        float4 a[4], b[4], c[4];
-        const int mb0 = c0 + tq;  // this warp's first token of the chunk
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (mb0 + j < m_valid)
-            a[j] = __ldcg(reinterpret_cast<const float4*>(lo_part + static_cast<size_t>(mb0 + j) * kTileRows));
-        int k = 0;
-        for (; k + 2 <= others; k += 2) {
-          const float* pb = next_part + k * stride;
-          const float* pc = pb + stride;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (mb0 + j < m_valid) {
-              b[j] = __ldcg(reinterpret_cast<const float4*>(pb + static_cast<size_t>(mb0 + j) * kTileRows));
-              c[j] = __ldcg(reinterpret_cast<const float4*>(pc + static_cast<size_t>(mb0 + j) * kTileRows));
-            }
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (mb0 + j < m_valid) {
-              a[j].x += b[j].x; a[j].y += b[j].y; a[j].z += b[j].z; a[j].w += b[j].w;
-              a[j].x += c[j].x; a[j].y += c[j].y; a[j].z += c[j].z; a[j].w += c[j].w;
-            }
-        }
-        if (k < others) {
-          const float* pb = next_part + k * stride;
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (mb0 + j < m_valid) {
-              b[j] = __ldcg(reinterpret_cast<const float4*>(pb + static_cast<size_t>(mb0 + j) * kTileRows));
-              a[j].x += b[j].x; a[j].y += b[j].y; a[j].z += b[j].z; a[j].w += b[j].w;
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = mb0 + j;
-          if (m >= m_valid) continue;
-          const float sx = m0 == staged_m0 ? bars->sx[m] : __ldg(p.s_x + m0 + m);
-          const uint32_t v0 = to_bf16_bits(a[j].x * sw[0] * sx), v1 = to_bf16_bits(a[j].y * sw[1] * sx);
-          const uint32_t v2 = to_bf16_bits(a[j].z * sw[2] * sx), v3 = to_bf16_bits(a[j].w * sw[3] * sx);
-          uint16_t* yrow = mb.y + static_cast<size_t>(m0 + m) * mb.ldy;
-          if (vec) {
-            *reinterpret_cast<uint2*>(yrow + n0) = make_uint2(v0 | (v1 << 16), v2 | (v3 << 16));
-          } else {
-            const uint32_t vv[4] = {v0, v1, v2, v3};
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (n0 + i < mb.N) yrow[n0 + i] = static_cast<uint16_t>(vv[i]);
-          }
-        }
-      }
-      if (et == 0) p.counters[t * P + prank] = 0u;  // re-arm for the next launch (ordered by the kernel boundary)
+      stage_sx((t % p.m_tiles) * p.npad);
+      fixup_tile(p, t, P, prank, et, 128, bars->sx);
     };
 
     // Tiles this CTA must finish. Their fix-ups wait until this CTA has
@@ -783,7 +818,8 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             uint32_t v[16];
             ptx::tmem_ld_32x32b_x16(lane_base + static_cast<uint32_t>(c0), v);
             ptx::tmem_ld_wait();
-            float a[16];
+            float a[16], s16[16];
+            load_sx16(bars->sx + c0, s16);
 #pragma unroll
             for (int i = 0; i < 16; ++i) a[i] = __uint_as_float(v[i]);
             for (int r = 1; r < p.cluster; ++r) {
@@ -801,7 +837,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
             if (vec) {
               if (c > 0) ptx::named_bar_sync(1, 128);  // the previous chunk's readers are done
 #pragma unroll
-              for (int i = 0; i < 16; ++i) ystage[i * kTileRows + row] = to_bf16_bits(a[i] * sw * bars->sx[c0 + i]);
+              for (int i = 0; i < 16; ++i) ystage[i * kTileRows + row] = to_bf16_bits(a[i] * sw * s16[i]);
               ptx::named_bar_sync(1, 128);
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
@@ -816,7 +852,7 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
               for (int i = 0; i < 16; ++i) {
                 const int m = c0 + i;
                 if (m < m_valid)
-                  mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] = to_bf16_bits(a[i] * sw * bars->sx[m]);
+                  mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] = to_bf16_bits(a[i] * sw * s16[i]);
               }
             }
           }
@@ -858,12 +894,32 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         ptx::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(c0), v);
         ptx::tmem_ld_wait();
         if (whole) {
-          if (row_ok) {
+          float s16[16];
+          load_sx16(bars->sx + c0, s16);
+          const int nw = n - lane;  // the warp's first row
+          if (wstage != nullptr && nw + 32 <= mb.N && (mb.ldy % 8) == 0) {
+            // The warp's 32 rows of the chunk go out as 16-byte stores through
+            // its 1 KB of staging, [16 tokens][32 rows] bf16 (one 2-byte store
+            // per row and token took about 5x as long for a 128-token tile).
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              wstage[i * 32 + lane] = to_bf16_bits(__uint_as_float(v[i]) * sw * s16[i]);
+            __syncwarp();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = lane + 32 * h;  // 16-byte piece: token q / 4, rows 8 (q % 4) .. 8 (q % 4) + 7
+              const int m = c0 + (q >> 2);
+              if (m < m_valid)
+                ptx::st_global_v4(mb.y + static_cast<size_t>(m0 + m) * mb.ldy + nw + 8 * (q & 3),
+                                  reinterpret_cast<const uint4*>(wstage)[q]);
+            }
+            __syncwarp();
+          } else if (row_ok) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int m = c0 + i;
               if (m < m_valid)
-                mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] = to_bf16_bits(__uint_as_float(v[i]) * sw * bars->sx[m]);
+                mb.y[static_cast<size_t>(m0 + m) * mb.ldy + n] = to_bf16_bits(__uint_as_float(v[i]) * sw * s16[i]);
             }
           }
         } else {
@@ -904,7 +960,15 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
         next_whole = (a2 == 0 && b2 == units.nblk_of(t2));
       }
       if (next_whole) {
-        for (int i = 0; i < npending; ++i) finish_tile(pending[i]);
+        if (u + 1 == units.count) {
+          // The CTA's last unit: its fix-ups run at the end with every warp.
+          if (et == 0) {
+            for (int i = 0; i < npending; ++i) bars->pend[i] = pending[i];
+            bars->npend = npending;
+          }
+        } else {
+          for (int i = 0; i < npending; ++i) finish_tile(pending[i]);
+        }
         npending = 0;
       }
     }
@@ -935,6 +999,21 @@ __global__ void __launch_bounds__(kGemmThreadsMax, 2)
       ptx::tmem_dealloc_pair(bars->tmem_base, p.tmem_cols);
     else
       ptx::tmem_dealloc(bars->tmem_base, p.tmem_cols);
+  }
+  // Stream-K fix-ups left from the CTA's last unit, with every warp (the
+  // loaders and the MMA warp are done): twice the loads in flight of the
+  // epilogue warps alone, on the kernel's tail.
+  const int npend = bars->npend;
+  if (npend > 0) {
+    ptx::griddep_wait();  // s_x and Y may belong to the previous grid (a no-op once it has completed)
+    for (int i = 0; i < npend; ++i) {
+      const int t = bars->pend[i];
+      const int m0 = (t % p.m_tiles) * p.npad;
+      if (i > 0) __syncthreads();  // the previous fix-up's readers of the scales are done
+      for (int k = threadIdx.x; k < p.npad; k += blockDim.x) bars->sx[k] = m0 + k < p.M ? __ldg(p.s_x + m0 + k) : 0.0f;
+      __syncthreads();
+      fixup_tile(p, t, P, prank, threadIdx.x, blockDim.x, bars->sx);
+    }
   }
   if (pair) {
     // Neither CTA of a pair leaves while the other may still signal into it:

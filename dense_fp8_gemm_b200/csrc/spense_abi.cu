@@ -452,7 +452,14 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
                                          block_at(i, ci - tl * pl.mem_cost[i]));
     }
   }
-  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes + pl.recv_bytes;
+  // Output staging for the stream-K epilogue's whole tiles (16-byte stores),
+  // when the ring leaves room for it.
+  {
+    const uint32_t budget = gemm_max_smem() / pl.ctas_per_sm - (pl.ctas_per_sm > 1 ? 1024u : 0u);
+    const uint32_t used = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes + pl.recv_bytes;
+    pl.ystage = (pl.cluster == 1 && used + kYStageBytes <= budget) ? kYStageBytes : 0u;
+  }
+  pl.smem_bytes = reserve + static_cast<uint32_t>(pl.stages) * pl.stage_bytes + pl.recv_bytes + pl.ystage;
   WorkspaceLayout& w = pl.ws;
   size_t off = 256;  // header: status word
   w.counters_off = off;
@@ -581,6 +588,7 @@ spense_status prepare_gemm(const spense_packed* const* hs, int count, const uint
   p.x_warp = x_warp();
   p.w_keep = w_keep_knob() >= 0 ? w_keep_knob() : (pl.m_tiles > 1 ? 1 : 0);
   p.pair = pl.pair;
+  p.ystage = pl.ystage;
 #ifdef SPENSE_TEST_HOOKS
   // Test build only: with SPENSE_TEST_STALL=1 the loaders wait on header word
   // 16 of the workspace, which nothing sets, so every launch ends by timeout.
@@ -1014,6 +1022,7 @@ spense_status spense_plan_shapes(int count, const int64_t* N, const int64_t* K, 
   out->recv_bytes = pl.recv_bytes;
   out->l2_prefetch = l2_prefetch_for(pl);
   out->pair = pl.pair;
+  out->y_stage_bytes = pl.ystage;
   out->total_blocks = pl.cta_start[pl.grid];
   out->workspace_bytes = pl.ws.total_device;
   for (int g = 0; g <= pl.grid; ++g) out->cta_start[g] = pl.cta_start[g];

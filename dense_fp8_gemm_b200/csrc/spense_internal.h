@@ -22,6 +22,7 @@ constexpr int kGemmThreads = 192;       // warp 0 loads, warp 1 issues MMAs, war
 constexpr int kGemmThreadsMax = 256;    // plus a second weight loader and an activation loader
 constexpr int kMaxStages = 12;
 constexpr uint32_t kBarrierBytes = 2048;  // mbarriers, flags and staged token scales
+constexpr uint32_t kYStageBytes = 4096;   // whole-tile output staging: 16 tokens x 32 rows bf16 per epilogue warp
 
 // Workspace layout: [header 256 B][counters][partials][gathered X][host staging]
 struct WorkspaceLayout {
@@ -64,6 +65,7 @@ struct GemmPlan {
   int cluster;
   uint32_t recv_bytes;
   int pair;        // 1: CTA pairs (tcgen05 cta_group::2) share 256-row MMAs; the work units are pairs
+  uint32_t ystage; // bytes of output staging after the barrier area (0 or kYStageBytes)
   int cta_start[kMaxGrid + 1];  // first linear block of each work unit (CTA, or pair); [grid] = total blocks
   WorkspaceLayout ws;
 };
@@ -108,6 +110,7 @@ struct GemmParams {
   int x_warp;                     // 1: a warp of its own issues the activation-tile loads
   int w_keep;                     // 1: weight copies use the evict-normal L2 policy (re-read by token tiles)
   int pair;                       // 1: pair mode (grid = 2 CTAs per work unit, cluster of 2, M = 256 MMAs)
+  uint32_t ystage;                // stream-K: 1 KB of output staging per epilogue warp after the barriers, or 0
 };
 
 // Kernels (defined in the .cu files).

@@ -66,7 +66,8 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("npad", "box_rows", "m_tiles", "n_tiles", "tiles", "ctas_per_sm",
                                               "cluster", "grid", "stages", "nacc")] + \
                [(n, ctypes.c_uint32) for n in ("tmem_cols", "smem_bytes", "stage_bytes", "recv_bytes")] + \
-               [("l2_prefetch", ctypes.c_int32), ("pair", ctypes.c_int32), ("total_blocks", ctypes.c_int64),
+               [("l2_prefetch", ctypes.c_int32), ("pair", ctypes.c_int32), ("y_stage_bytes", ctypes.c_uint32),
+                ("total_blocks", ctypes.c_int64),
                 ("workspace_bytes", ctypes.c_uint64), ("cta_start", ctypes.c_int32 * (PLAN_MAX_GRID + 1))]
 
 

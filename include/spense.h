@@ -433,6 +433,7 @@ typedef struct spense_plan_info {
   uint32_t recv_bytes;   /* cluster mode: rank 0's area for the peers' partials */
   int32_t l2_prefetch;   /* weight blocks per CTA prefetched into L2 at start */
   int32_t pair;          /* 1: CTA pairs share 256-row MMAs; grid, n_tiles and cta_start then count pairs */
+  uint32_t y_stage_bytes; /* stream-K: shared memory staging whole output tiles for 16-byte stores (0: none) */
   int64_t total_blocks;  /* blocks the launch streams */
   uint64_t workspace_bytes;                    /* spense_gemm_grouped_workspace_size */
   int32_t cta_start[SPENSE_PLAN_MAX_GRID + 1]; /* [grid] = total_blocks */

@@ -88,7 +88,9 @@ def test_plan_invariants(name, M):
     xrows = npad // 2 if pair else npad  # token rows of a stage's activation tile in this CTA
     assert p["stage_bytes"] == 16384 + xrows * (256 if any_sparse else 128) + (4096 if any_sparse else 0)
     assert p["stages"] >= 2
-    assert p["smem_bytes"] == RESERVE + p["stages"] * p["stage_bytes"] + p["recv_bytes"]
+    assert p["smem_bytes"] == RESERVE + p["stages"] * p["stage_bytes"] + p["recv_bytes"] + p["y_stage_bytes"]
+    # whole-tile output staging (1 KB per epilogue warp) only for stream-K, and only where the ring leaves room
+    assert p["y_stage_bytes"] in (0, 4096) and (S == 1 or p["y_stage_bytes"] == 0)
     assert p["smem_bytes"] <= SMEM_MAX // cps - (1024 if cps > 1 else 0)
     # tensor memory: a power of two from 32 columns holding the accumulators and the metadata
     assert p["tmem_cols"] in (32, 64, 128, 256, 512)
