@@ -230,7 +230,9 @@ int bulk_split() {
 // of X: either none has a scattered dense set (their Kd may differ, e.g. the
 // 2:4 rows and the dense rows of an output-split weight), or all have the
 // same one.
-spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, int sms, GemmPlan* out) {
+// t_force: token tile to plan with (0: automatic; SPENSE_TOKEN_TILE overrides both).
+spense_status make_plan_t(const spense_packed* const* hs, int count, int64_t M, int sms, int t_force,
+                          GemmPlan* out) {
   if (hs == nullptr || count < 1 || count > kMaxGroup)
     return fail(SPENSE_ERR_ARG, "a launch takes 1 to %d packed weights, got %d", kMaxGroup, count);
   if (M < 1 || M > 65535) return fail(SPENSE_ERR_SHAPE, "M = %lld outside [1, 65535]", (long long)M);
@@ -257,10 +259,10 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   // weight rows, and token tiles of up to 256 tokens read each weight once.
   const int pk = pair_knob();
   pl.pair = (x_warp() && (pk == 2 || (pk == 1 && M > 64))) ? 1 : 0;
-  int T = token_tile_knob() != 0
-              ? token_tile_knob()
-              : (pl.pair ? kMaxTokenTile
-                         : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128));
+  int T = token_tile_knob() != 0 ? token_tile_knob()
+          : t_force != 0          ? t_force
+          : (pl.pair ? kMaxTokenTile
+                     : ((tiles64 <= sms || (tiles64 <= 2LL * sms && small_weight)) ? 64 : 128));
   // Tiles of 128 tokens that leave most CTAs straddling two tiles (fewer than
   // 1.5 tiles per SM) while tiles of 96 would give each about two: take 96
   // (q/k/v 12288x5120 at 256 tokens 35.3 -> 28.4 us; weights that stay at
@@ -484,6 +486,19 @@ spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, in
   for (int i = 0; i < count; ++i) off += round_up(static_cast<size_t>(M * hs[i]->N) * 2, 256);
   w.total_host = off;
   *out = pl;
+  return SPENSE_OK;
+}
+
+spense_status make_plan(const spense_packed* const* hs, int count, int64_t M, int sms, GemmPlan* out) {
+  const spense_status st = make_plan_t(hs, count, M, sms, 0, out);
+  if (st != SPENSE_OK) return st;
+  // Tiles of 64 tokens are chosen above 64 tokens so that the tiles can split
+  // over clusters; when no cluster split fits (long tiles, see cluster_for),
+  // tiles of 128 tokens halve the weight re-reads instead: down 5120x27648 at
+  // 128 tokens 38.6 -> 30.2 us, o_proj 5120x10240 21.6 -> 21.2 us.
+  if (token_tile_knob() == 0 && !out->pair && out->npad == 64 && M > 64 && out->cluster == 1 &&
+      static_cast<long long>(out->n_tiles) * ((M + 63) / 64) <= sms)
+    return make_plan_t(hs, count, M, sms, 128, out);
   return SPENSE_OK;
 }
 

@@ -110,7 +110,8 @@ def test_plan_invariants(name, M):
     ("gateup", 128, 128, 1, 1, 0), # many tiles: token tiles of 128
     ("down", 256, 128, 1, 1, 0),   # a 94 MB weight with 160 tiles of 64: tiles of 128
     ("q", 256, 64, 1, 1, 0),       # a 30 MB weight: its repeated reads stay in L2, tiles of 64
-    ("down36", 128, 64, 1, 1, 0),  # 135 blocks per tile: no two-stage cluster ring, stream-K with a deep one
+    ("down36", 128, 128, 1, 1, 0), # 135 blocks per tile: no cluster split fits, so one token tile, not two of 64
+    ("o36", 128, 128, 1, 1, 0),    # the same for o_proj (its tiles of 64 would be split over no cluster either)
     ("o36", 16, 16, 4, 2, 0),      # three stages at two CTAs per SM: clusters of 4 stay
     ("qkv36", 256, 96, 1, 1, 0),   # 128-token tiles: 1.3 per SM; 96: about 2 (45 MB stays in L2)
     ("down36", 600, 128, 1, 1, 0), # 102 MB: its re-reads would leave L2, tiles of 128 stay
