@@ -136,6 +136,30 @@ def test_gemm_matches_oracle(M, N, K, Kd, scattered):
     _assert_close(Y, yref, bound, f"M={M} N={N} K={K} Kd={Kd}")
 
 
+@pytest.mark.parametrize("pad", [3, 4, 8])
+def test_strided_outputs_keep_their_padding(pad):
+    # Outputs as column slices of a wider buffer (row stride N + pad elements), a ragged last row tile and
+    # token counts with whole and shared stream-K tiles: whole tiles go out as 16-byte stores only when the
+    # stride is a multiple of 8 elements and a warp's 32 rows are all in range, else as 2-byte stores; the
+    # padding columns must stay untouched either way.
+    # N = 40 x 128 + 104: 70 tokens split tiles over clusters of 2, 200 and 300 tokens run stream-K
+    N, K, Kd = 5224, 1024, 256
+    X0, s_x0, W, s_w, _ = _make(4242 + pad, 300, N, K, Kd)
+    ref = oracle.pack(W, Kd=Kd)
+    pw = spense.pack(_dev(W), _dev(s_w), Kd=Kd)
+    for M in (70, 200, 300):
+        X, s_x = X0[:M], s_x0[:M]
+        yref, bound = oracle.gemm(X, s_x, W, s_w, keep=ref["keep"])
+        big = torch.full((M, N + pad), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ws = spense.new_workspace(spense.grouped_workspace_size([pw], M))
+        spense.gemm_grouped([pw], _dev(X), _dev(s_x), Ys=[big[:, :N]], workspace=ws)
+        torch.cuda.synchronize()
+        assert spense.workspace_status(ws) == 0
+        _assert_close(big[:, :N], yref, bound, f"ldy={N + pad} M={M}")
+        assert torch.isnan(big[:, N:]).all(), "a store reached the padding columns"
+    pw.free()
+
+
 def test_gemm_with_explicit_mask():
     M, N, K, Kd = 12, 384, 1024, 256
     X, s_x, W, s_w, _ = _make(21, M, N, K, Kd)
