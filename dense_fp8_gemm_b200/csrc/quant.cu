@@ -164,11 +164,15 @@ cudaError_t launch_quantize(const uint16_t* X, int64_t M, int64_t K, const int32
   if (M == 0) return cudaSuccess;
   // CTAs per row: one once the rows alone cover the SMs (every extra CTA of a
   // row reads the row again); otherwise enough for two CTAs per SM, at most 8
-  // and at most one per 16-column chunk. Measured at 25600 columns, back to
-  // back: 1, 2, 4, 8, 16 CTAs per row take 7.8, 6.3, 4.7, 3.8, 3.5 us at 16
-  // tokens and 8.5, 6.8, 4.8, 4.0, 6.6 us at 32 tokens.
+  // (16 for a gather at 4 to 16 tokens) and at most one per 16-column chunk.
+  // Measured at 25600 columns, back to back: 1, 2, 4, 8, 16 CTAs per row take
+  // 7.8, 6.3, 4.7, 3.8, 3.5 us at 16 tokens and 8.5, 6.8, 4.8, 4.0, 6.6 us at
+  // 32 tokens; with the gather 16 rather than 8 per row: 3.61 -> 3.40 us at 4
+  // tokens, 3.82 -> 3.55 at 16, but 2.96 -> 3.21 at one token, and without the
+  // gather no gain (3.28 -> 3.36 at 16).
   int64_t C = M >= sms ? 1 : (2 * static_cast<int64_t>(sms) + M - 1) / M;
-  C = C < 1 ? 1 : (C > 8 ? 8 : C);
+  const int64_t cmax = (perm != nullptr && M >= 4 && M <= 16) ? 16 : 8;
+  C = C < 1 ? 1 : (C > cmax ? cmax : C);
 
   while (C > 1 && K / 16 < C) --C;
   const unsigned int grid = static_cast<unsigned int>(M * C);
